@@ -1,0 +1,207 @@
+/*
+ * libvlaq — NVFP4 / FP8 quantize + linear for one NVIDIA B200 (sm_100a).
+ *
+ * The quantized linear projection of a VLA language backbone:
+ *   1. dynamic per-token NVFP4 activation quantization, optionally after a
+ *      fused RMSNorm and a block-64 Walsh-Hadamard rotation;
+ *   2. a block-scaled FP4 GEMM against offline NVFP4 weights, BF16 output,
+ *      optional fused residual add;
+ *   3. an FP8 E4M3 W8A8 variant (per-row weight scale, per-token activation
+ *      scale).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Device pointers are CUDA global-memory pointers of the current device;
+ *   all of them must be 16-byte aligned (TMA and 128-bit accesses).
+ *   "stream" is a cudaStream_t (NULL = legacy default stream).
+ * - bf16 tensors are row-major with unit stride along K.
+ * - The caller allocates every buffer (outputs and workspace).  The library
+ *   never allocates device memory and keeps no state between calls except a
+ *   thread-local error string and a device status word.
+ * - Every call validates its arguments on the host first.  On any error it
+ *   returns a non-zero vlaq_status, sets vlaq_last_error(), launches nothing
+ *   and touches no output.  Otherwise the work is queued on `stream` and the
+ *   call returns VLAQ_OK without synchronizing.
+ * - A kernel whose bounded internal wait runs out records VLAQ_ERR_TIMEOUT
+ *   in the device status word and returns; vlaq_check() reports it.
+ *
+ * Data formats
+ * ------------
+ * NVFP4 ("Feat/internvla n1 dualvln", NVFP4 loader and nibble-order commits;
+ * "Alpamayo 2 Super NVFP4" test reflection, ModelOpt configuration):
+ *   value = E2M1(code) * E4M3(block scale) * g       (block = 16 along K)
+ *   g = amax / (6 * 448): one fp32 per token row for activations, one per
+ *   tensor for weights.  Block scale = E4M3_rne_sat(a_b / (6 g)); code =
+ *   E2M1_rne_sat(x / (E4M3(scale) * g)); all fp32 with correctly rounded
+ *   division.  g == 0 gives zero scales and codes.
+ *
+ *   Packed codes: row r, element k lives in byte r * pitch + k / 2, in the
+ *   low nibble when k is even.  pitch = vlaq_nvfp4_code_pitch(K) =
+ *   ceil(K / 64) * 32 bytes (= K / 2 whenever K % 64 == 0); bytes past K / 2
+ *   in a row are written as zero.
+ *
+ *   Block scales, 128x4 tiled (the layout the tensor cores read, so no
+ *   second copy is ever needed): rows are padded to Rp = ceil(rows/128)*128,
+ *   scale columns to Cp = ceil(K/64)*4.  The scale of row r, block j
+ *   (j = k / 16) is the byte at
+ *       ((r / 128) * (Cp / 4) + j / 4) * 512
+ *       + (r % 32) * 16 + ((r % 128) / 32) * 4 + (j % 4).
+ *   Total size vlaq_nvfp4_scale_bytes(rows, K) = Rp * Cp.  Padded columns
+ *   (j >= K/16) of real rows are written as zero; padded rows are never
+ *   written and never affect a stored output.
+ *
+ * FP8 E4M3 (per-row scale):  value = E4M3(code) * s,  s = amax / 448.
+ *   Codes row-major [rows, K], one byte per element.
+ *
+ * Optional activation transforms (flags), applied before the amax:
+ *   VLAQ_F_RMSNORM    y = (x * r) * gamma, r = 1 / sqrt(mean(x^2) + eps),
+ *                     fp32; the sum of squares uses 32 lanes, lane l owning
+ *                     the 8-element chunks l, l+32, ... in element order,
+ *                     combined by an XOR butterfly 16, 8, 4, 2, 1
+ *                     ("FoldQuant W8A8/W4A4 inference", SYCL commit).
+ *   VLAQ_F_HADAMARD64 block-diagonal normalised Sylvester Walsh-Hadamard
+ *                     transform, block 64 (same page, dequant commit); needs
+ *                     K % 64 == 0.
+ */
+#ifndef VLAQ_H_
+#define VLAQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define VLAQ_API __attribute__((visibility("default")))
+#else
+#define VLAQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VLAQ_OK = 0,
+  VLAQ_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad flag      */
+  VLAQ_ERR_SHAPE = 2,       /* K not divisible by 16 (64 with Hadamard),  */
+                            /* or a size beyond a documented limit        */
+  VLAQ_ERR_ALIGN = 3,       /* a pointer not 16-byte aligned               */
+  VLAQ_ERR_ARCH = 4,        /* current device is not sm_100               */
+  VLAQ_ERR_CUDA = 5,        /* a CUDA runtime / driver call failed         */
+  VLAQ_ERR_TIMEOUT = 6,     /* a device-side bounded wait ran out          */
+  VLAQ_ERR_WORKSPACE = 7    /* workspace missing or smaller than needed    */
+} vlaq_status;
+
+enum {
+  VLAQ_F_RMSNORM = 1u << 0,
+  VLAQ_F_HADAMARD64 = 1u << 1
+};
+
+/* Human-readable text of the last error on the calling thread ("" if
+ * none).  A K that is not a multiple of 16 reports the division, e.g.
+ * "... 3420 / 16 = 213.75 ..." ("Feat/internvla n1 dualvln", scheme gate).
+ * The pointer stays valid until the next vlaq call on this thread. */
+VLAQ_API const char* vlaq_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+VLAQ_API int vlaq_version(void);
+
+/* Synchronizes `stream`, then reads and clears the device status word of
+ * the current device.  Returns VLAQ_ERR_TIMEOUT if a kernel gave up a
+ * bounded wait since the last check, VLAQ_ERR_CUDA on a CUDA error. */
+VLAQ_API vlaq_status vlaq_check(void* stream);
+
+/* ----------------------------------------------------------- size helpers */
+VLAQ_API int64_t vlaq_nvfp4_code_pitch(int64_t K);               /* bytes per row   */
+VLAQ_API int64_t vlaq_nvfp4_scale_bytes(int64_t rows, int64_t K);/* tiled scales    */
+
+/* ------------------------------------------------------------------ NVFP4 */
+
+/* Offline weight quantization, one global scale for the whole tensor.
+ *   W       bf16 [N, K] (device)
+ *   flags   0 or VLAQ_F_HADAMARD64 (rotate each row before quantizing)
+ *   codes   out, vlaq_nvfp4_code_pitch(K) * N bytes
+ *   scales  out, vlaq_nvfp4_scale_bytes(N, K) bytes (128x4 tiled)
+ *   g_w     out, one fp32
+ * Limits: 1 <= N, 16 <= K <= 32768, K % 16 == 0.
+ * ("Alpamayo 2 Super NVFP4": max calibration, FP4 weights, block 16, FP8
+ * block scales; "Feat/internvla n1 dualvln": float32 global scale.) */
+VLAQ_API vlaq_status vlaq_quantize_weight_nvfp4(const void* W, int64_t N, int64_t K,
+                                       uint32_t flags, uint8_t* codes,
+                                       uint8_t* scales, float* g_w,
+                                       void* stream);
+
+/* Dynamic per-token activation quantization (the fused prologue).
+ *   X       bf16 [M, K] (device)
+ *   gamma   bf16 [K] RMSNorm gain (device), required with VLAQ_F_RMSNORM,
+ *           else ignored (may be NULL)
+ *   eps     RMSNorm epsilon (e.g. 1e-6)
+ *   flags   any of VLAQ_F_RMSNORM | VLAQ_F_HADAMARD64
+ *   codes   out, vlaq_nvfp4_code_pitch(K) * M bytes
+ *   scales  out, vlaq_nvfp4_scale_bytes(M, K) bytes (128x4 tiled)
+ *   g_x     out, M fp32 (one global scale per token)
+ * M == 0 is a no-op.  Limits: 16 <= K <= 32768, K % 16 == 0.
+ * ("NVIDIA/TensorRT-Edge-LLM PR #193": NVFP4 quantizes activations
+ * dynamically; "FoldQuant W8A8/W4A4 inference": RMSNorm + butterfly + quant
+ * prologue with per-token amax, round-half-even and clamp.) */
+VLAQ_API vlaq_status vlaq_quantize_act_nvfp4(const void* X, int64_t M, int64_t K,
+                                    const void* gamma, float eps,
+                                    uint32_t flags, uint8_t* codes,
+                                    uint8_t* scales, float* g_x,
+                                    void* stream);
+
+/* Bytes of fp32 workspace vlaq_linear_nvfp4 / vlaq_linear_fp8 need for the
+ * given shape on the current device (0 when the shape runs without split-K).
+ * The workspace holds per-split partial sums; its contents on entry do not
+ * matter. */
+VLAQ_API size_t vlaq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* Y = bf16_rne( (sum_k dec(x)[m,k] * dec(w)[n,k]) + residual[m,n] )
+ * with the product accumulated in fp32 on the tensor cores
+ * (tcgen05 kind::mxf4nvf4, block-16 E4M3 scales) and the global scales
+ * g_x[m] * g_w applied in the epilogue.
+ *   xq, xs, g_x  activation codes / tiled scales / globals (M rows)
+ *   wq, ws, g_w  weight codes / tiled scales / global (N rows)
+ *   residual     bf16 [M, N] or NULL
+ *   Y            out, bf16 [M, N]
+ *   workspace    device buffer of ws_bytes >= vlaq_linear_workspace_bytes
+ * M == 0 is a no-op.  Limits: 1 <= N, 16 <= K, K % 16 == 0, N % 8 == 0.
+ * (Residual add in the o / down epilogues: "FoldQuant W8A8/W4A4 inference",
+ * merge commit.) */
+VLAQ_API vlaq_status vlaq_linear_nvfp4(const uint8_t* xq, const uint8_t* xs,
+                              const float* g_x, const uint8_t* wq,
+                              const uint8_t* ws, const float* g_w,
+                              const void* residual, void* Y, int64_t M,
+                              int64_t N, int64_t K, void* workspace,
+                              size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------ FP8 W8A8 */
+
+/* Per-row weight quantization: s_w[n] = max|w_n| / 448, codes E4M3.
+ *   W bf16 [N, K]; flags 0 or VLAQ_F_HADAMARD64; codes out [N, K];
+ *   s_w out, N fp32.  Limits: 16 <= K <= 32768, K % 16 == 0. */
+VLAQ_API vlaq_status vlaq_quantize_weight_fp8(const void* W, int64_t N, int64_t K,
+                                     uint32_t flags, uint8_t* codes,
+                                     float* s_w, void* stream);
+
+/* Per-token activation quantization with the same optional RMSNorm /
+ * Hadamard prologue as the NVFP4 variant.  codes out [M, K]; s_x out, M
+ * fp32.  ("Feat/internvla n1 dualvln": FP8 E4M3 weight + scale tensors.) */
+VLAQ_API vlaq_status vlaq_quantize_act_fp8(const void* X, int64_t M, int64_t K,
+                                  const void* gamma, float eps,
+                                  uint32_t flags, uint8_t* codes, float* s_x,
+                                  void* stream);
+
+/* Y = bf16_rne( s_x[m] * s_w[n] * sum_k e4m3(x)[m,k] e4m3(w)[n,k]
+ *               + residual[m,n] ), fp32 accumulation on the tensor cores
+ * (tcgen05 kind::f8f6f4).  Same argument rules as vlaq_linear_nvfp4. */
+VLAQ_API vlaq_status vlaq_linear_fp8(const uint8_t* xq, const float* s_x,
+                            const uint8_t* wq, const float* s_w,
+                            const void* residual, void* Y, int64_t M,
+                            int64_t N, int64_t K, void* workspace,
+                            size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VLAQ_H_ */

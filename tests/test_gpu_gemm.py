@@ -1,0 +1,132 @@
+"""GPU parity of the tcgen05 GEMMs against the fp64 oracle.
+
+The GEMM is fed the oracle's own codes and scales (re-laid out into the
+library's padded / tiled buffers), so the comparison isolates the GEMM; the
+end-to-end cases run the GPU quantizers too (their bytes are bit-exact, see
+test_gpu_quant.py).  Gate: relative Frobenius error < 2e-3 against the fp64
+result on the same decoded operands; max-abs is reported."""
+import numpy as np
+import pytest
+import torch
+
+import layouts
+import oracle
+import synthetic_inputs as si
+from gpu_helpers import (REL_FRO_TOL, bits, gemm_error, gpu_linear_fp8, gpu_linear_nvfp4,
+                         gpu_quant_act_nvfp4, gpu_quant_weight_nvfp4, to_dev, vq)
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_case(M, N, K, seed, residual=False, flags=0):
+    X = si.projection_activations(K, M, seed)
+    W = si.projection_weight(K, N, seed)
+    cx, sx, gx = oracle.quantize_nvfp4(bits(X), flags=flags)
+    cw, sw, gw = oracle.quantize_nvfp4(bits(W), flags=flags, per_tensor=True)
+    R = si.residual(M, N, seed) if residual else None
+    dx = oracle.decode_nvfp4(cx, sx, gx, K)
+    dw = oracle.decode_nvfp4(cw, sw, gw, K, per_tensor=True)
+    Y64 = oracle.linear_f64(dx, dw, None if R is None else bits(R))
+    return (cx, sx, gx, cw, sw, gw, R, Y64)
+
+
+def _run_nvfp4_from_oracle(M, N, K, case):
+    cx, sx, gx, cw, sw, gw, R, _ = case
+    return gpu_linear_nvfp4(to_dev(layouts.pad_codes(cx, K)), to_dev(layouts.tile_scales(sx, M, K)), to_dev(gx),
+                            to_dev(layouts.pad_codes(cw, K)), to_dev(layouts.tile_scales(sw, N, K)), to_dev(gw),
+                            M, N, K, None if R is None else R.cuda())
+
+
+# (M, N, K): one tile; ragged M / N / K tails; several K stages; split-K
+# decode shapes (M <= 8 with few N tiles); residual add.
+NVFP4_CASES = [
+    (16, 128, 256, False),
+    (128, 128, 256, False),
+    (300, 392, 1024, False),
+    (130, 264, 336, True),
+    (257, 136, 3584, True),
+    (1, 512, 4096, False),
+    (4, 256, 2048, True),
+    (8, 1024, 3584, False),
+    (1, 8, 64, False),
+    (64, 4608, 256, False),
+]
+
+
+@pytest.mark.parametrize("M,N,K,res", NVFP4_CASES)
+def test_linear_nvfp4_vs_oracle(M, N, K, res):
+    case = _oracle_case(M, N, K, 21, residual=res)
+    Y = _run_nvfp4_from_oracle(M, N, K, case)
+    rel, mx = gemm_error(Y, case[-1])
+    print(f"nvfp4 M={M} N={N} K={K} res={res}: rel_fro={rel:.3e} max_abs={mx:.3e}")
+    assert rel < REL_FRO_TOL, (rel, mx)
+
+
+def test_linear_nvfp4_single_element_parity_positions():
+    """1x16x1-style probe: one non-zero element at every position of a
+    16-block (both nibbles, every k-step) must land on the right product."""
+    M, N, K = 1, 8, 256
+    for pos in range(0, K, 7):
+        x = np.zeros((M, K), np.float32)
+        w = np.zeros((N, K), np.float32)
+        x[0, pos] = 3.0
+        w[:, pos] = np.arange(1, N + 1, dtype=np.float32)
+        Xb = torch.from_numpy(x).to(torch.bfloat16)
+        Wb = torch.from_numpy(w).to(torch.bfloat16)
+        cx, sx, gx = oracle.quantize_nvfp4(bits(Xb))
+        cw, sw, gw = oracle.quantize_nvfp4(bits(Wb), per_tensor=True)
+        Y64 = oracle.linear_f64(oracle.decode_nvfp4(cx, sx, gx, K),
+                                oracle.decode_nvfp4(cw, sw, gw, K, per_tensor=True))
+        Y = _run_nvfp4_from_oracle(M, N, K, (cx, sx, gx, cw, sw, gw, None, Y64))
+        rel, _ = gemm_error(Y, Y64)
+        assert rel < REL_FRO_TOL, (pos, rel)
+
+
+@pytest.mark.parametrize("M,N,K,res", [(16, 128, 256, False), (300, 392, 1024, True), (129, 136, 208, False),
+                                       (1, 512, 4096, True), (8, 256, 2048, False), (257, 264, 3584, False)])
+def test_linear_fp8_vs_oracle(M, N, K, res):
+    X = si.projection_activations(K, M, 31)
+    W = si.projection_weight(K, N, 31)
+    cx, sx = oracle.quantize_fp8(bits(X))
+    cw, sw = oracle.quantize_fp8(bits(W))
+    R = si.residual(M, N, 31) if res else None
+    Y64 = oracle.linear_f64(oracle.decode_fp8(cx, sx), oracle.decode_fp8(cw, sw), None if R is None else bits(R))
+    Y = gpu_linear_fp8(to_dev(cx), to_dev(sx), to_dev(cw), to_dev(sw), M, N, K, None if R is None else R.cuda())
+    rel, mx = gemm_error(Y, Y64)
+    print(f"fp8 M={M} N={N} K={K}: rel_fro={rel:.3e} max_abs={mx:.3e}")
+    assert rel < REL_FRO_TOL, (rel, mx)
+
+
+@pytest.mark.parametrize("M,N,K,flags,res", [(200, 256, 1024, 0, False), (70, 384, 512, 3, True),
+                                             (3, 640, 2048, 2, True)])
+def test_end_to_end_nvfp4(M, N, K, flags, res):
+    """GPU quantizers + GPU GEMM vs oracle quantizers + fp64 GEMM."""
+    m = vq()
+    X = si.projection_activations(K, M, 41)
+    W = si.projection_weight(K, N, 41)
+    gam = si.norm_gain(K, 41)
+    R = si.residual(M, N, 41) if res else None
+    cx, sx, gx = oracle.quantize_nvfp4(bits(X), bits(gam), 1e-6, flags)
+    cw, sw, gw = oracle.quantize_nvfp4(bits(W), flags=flags & 2, per_tensor=True)
+    Y64 = oracle.linear_f64(oracle.decode_nvfp4(cx, sx, gx, K), oracle.decode_nvfp4(cw, sw, gw, K, per_tensor=True),
+                            None if R is None else bits(R))
+    xq, xs, xg = m.alloc_nvfp4(M, K)
+    wq, ws, wg = m.alloc_nvfp4(N, K, per_tensor=True)
+    m.vlaq_quantize_weight_nvfp4(W.cuda(), N, K, flags & 2, wq, ws, wg)
+    m.vlaq_quantize_act_nvfp4(X.cuda(), M, K, gam.cuda(), 1e-6, flags, xq, xs, xg)
+    Y = gpu_linear_nvfp4(xq, xs, xg, wq, ws, wg, M, N, K, None if R is None else R.cuda())
+    rel, mx = gemm_error(Y, Y64)
+    assert rel < REL_FRO_TOL, (rel, mx)
+
+
+def test_workspace_is_checked():
+    m = vq()
+    M, N, K = 1, 512, 4096
+    need = m.vlaq_linear_workspace_bytes(M, N, K)
+    assert need > 0  # this decode shape runs split-K
+    xq, xs, xg = m.alloc_nvfp4(M, K)
+    wq, ws, wg = m.alloc_nvfp4(N, K, per_tensor=True)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(m.VlaqError) as ei:
+        m.vlaq_linear_nvfp4(xq, xs, xg, wq, ws, wg, None, Y, M, N, K, None, 0)
+    assert ei.value.status == 7

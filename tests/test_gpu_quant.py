@@ -1,0 +1,101 @@
+"""GPU parity of the quantizers: bit-exact codes, block scales and global
+scales against the CPU oracle on the same seeded bf16 inputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic_inputs as si
+from gpu_helpers import (assert_nvfp4_equal, bits, gpu_quant_act_nvfp4, gpu_quant_fp8,
+                         gpu_quant_weight_nvfp4)
+
+pytestmark = pytest.mark.gpu
+
+# (M, K): several 64-blocks per row, ragged K % 64 in {16, 32, 48}, multiple
+# 128-row tiles with a ragged tail, the minimum K and the maximum supported K.
+SHAPES = [(16, 256), (1, 16), (3, 48), (130, 336), (257, 1024), (64, 3584), (5, 18944), (2, 32768),
+          (129, 96)]
+
+
+def _inputs(M, K, seed):
+    X = si.projection_activations(K, M, seed)
+    return X
+
+
+@pytest.mark.parametrize("M,K", SHAPES)
+def test_act_nvfp4_plain(M, K):
+    X = _inputs(M, K, 7)
+    ref = oracle.quantize_nvfp4(bits(X))
+    assert_nvfp4_equal(gpu_quant_act_nvfp4(X), ref, M, K, f"act {M}x{K}")
+
+
+@pytest.mark.parametrize("M,K", [(s[0], s[1]) for s in SHAPES if s[1] % 64 == 0])
+@pytest.mark.parametrize("flags", [1, 2, 3])
+def test_act_nvfp4_norm_hadamard(M, K, flags):
+    X = _inputs(M, K, 8)
+    gam = si.norm_gain(K, 8)
+    ref = oracle.quantize_nvfp4(bits(X), bits(gam), 1e-6, flags)
+    assert_nvfp4_equal(gpu_quant_act_nvfp4(X, gam, 1e-6, flags), ref, M, K, f"act {M}x{K} f{flags}")
+
+
+def test_act_nvfp4_rmsnorm_ragged_k():
+    X = _inputs(33, 336, 9)
+    gam = si.norm_gain(336, 9)
+    ref = oracle.quantize_nvfp4(bits(X), bits(gam), 1e-5, 1)
+    assert_nvfp4_equal(gpu_quant_act_nvfp4(X, gam, 1e-5, 1), ref, 33, 336, "rmsnorm K=336")
+
+
+def test_act_nvfp4_tiny_config_outliers():
+    X, _ = si.tiny_inputs(0)
+    ref = oracle.quantize_nvfp4(bits(X))
+    assert_nvfp4_equal(gpu_quant_act_nvfp4(X), ref, 16, 256, "tiny")
+
+
+def test_act_nvfp4_edge_values():
+    """Zero rows, negative zeros, rounding ties, tiny and huge magnitudes."""
+    K = 256
+    rows = []
+    rows.append(np.zeros(K, np.float32))                                   # all-zero row: g = 0
+    r = np.zeros(K, np.float32); r[::2] = -0.0; r[7] = 6.0; rows.append(r)  # -0 next to a max
+    # grid midpoints relative to amax 6 -> ties in x / S
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0], np.float32)
+    r = np.tile(np.concatenate([mids, -mids]), K // 16).astype(np.float32); rows.append(r)
+    r = np.full(K, 1e-38, np.float32); r[3] = 3e-38; rows.append(r)         # subnormal-ish scales
+    r = np.full(K, 3e38, np.float32); r[5] = -3.3e38; rows.append(r)        # near bf16 max
+    r = np.zeros(K, np.float32); r[100] = 1e-3; r[200] = 1e3; rows.append(r)  # mixed block scales
+    rng = np.random.default_rng(3)
+    r = (rng.standard_normal(K) * np.exp2(rng.integers(-30, 30, K))).astype(np.float32); rows.append(r)
+    X = torch.from_numpy(np.stack(rows)).to(torch.bfloat16)
+    ref = oracle.quantize_nvfp4(bits(X))
+    assert_nvfp4_equal(gpu_quant_act_nvfp4(X), ref, X.shape[0], K, "edge values")
+
+
+@pytest.mark.parametrize("N,K,flags", [(128, 256, 0), (300, 1024, 2), (37, 336, 0), (1, 64, 2),
+                                       (513, 3584, 0)])
+def test_weight_nvfp4(N, K, flags):
+    W = si.projection_weight(K, N, 11)
+    ref = oracle.quantize_nvfp4(bits(W), flags=flags, per_tensor=True)
+    assert_nvfp4_equal(gpu_quant_weight_nvfp4(W, flags), ref, N, K, f"weight {N}x{K} f{flags}")
+
+
+@pytest.mark.parametrize("M,K", SHAPES)
+@pytest.mark.parametrize("flags", [0, 3])
+def test_act_fp8(M, K, flags):
+    if flags and K % 64:
+        pytest.skip("Hadamard needs K % 64 == 0")
+    X = _inputs(M, K, 12)
+    gam = si.norm_gain(K, 12)
+    rc, rs = oracle.quantize_fp8(bits(X), bits(gam), 1e-6, flags)
+    gc, gs = gpu_quant_fp8(X, gam, 1e-6, flags)
+    bad = np.argwhere(gc != rc)
+    assert bad.size == 0, f"{len(bad)} fp8 codes differ, first {bad[:4].tolist()}"
+    assert np.array_equal(gs.view(np.uint32), rs.view(np.uint32))
+
+
+@pytest.mark.parametrize("N,K,flags", [(128, 256, 0), (77, 1024, 2), (40, 208, 0)])
+def test_weight_fp8(N, K, flags):
+    W = si.projection_weight(K, N, 13)
+    rc, rs = oracle.quantize_fp8(bits(W), flags=flags)
+    gc, gs = gpu_quant_fp8(W, flags=flags, weight=True)
+    assert np.array_equal(gc, rc)
+    assert np.array_equal(gs.view(np.uint32), rs.view(np.uint32))

@@ -1,0 +1,574 @@
+// Block-scaled FP4 (NVFP4) and FP8 E4M3 GEMM on the sm_100a tensor cores.
+//
+//   Y[m, n] = bf16_rne( acc[m, n] * scale(m, n) + residual[m, n] )
+//   acc[m, n] = sum_b sx[m, b] sw[n, b] sum_{k in b} e2m1(x[m, k]) e2m1(w[n, k])   (NVFP4)
+//             = sum_k e4m3(x[m, k]) e4m3(w[n, k])                                 (FP8)
+//   scale = g_x[m] * g_w (NVFP4) or s_x[m] * s_w[n] (FP8)
+//
+// Persistent, warp-specialised kernel, one CTA per SM:
+//   warp 0      TMA producer: 2-D tiled loads of the packed codes (128-byte
+//               swizzle) and 1-D bulk loads of the 512-byte scale atoms into
+//               a ring of shared-memory stages;
+//   warp 1      allocates TMEM and issues, from one thread, tcgen05.cp of the
+//               scale atoms into TMEM and tcgen05.mma (kind::mxf4nvf4 with
+//               block-16 UE4M3 scale vectors, or kind::f8f6f4) accumulating
+//               a 128 x BN fp32 tile in TMEM; tcgen05.commit frees stages
+//               and hands finished accumulators to the epilogue;
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (double-buffered in
+//               TMEM so the next tile's MMAs overlap), scale, residual add,
+//               bf16 round, 16-byte global stores.
+// Split-K (decode shapes, few output tiles): each split writes fp32 partial
+// sums to the caller's workspace and a small kernel reduces them in fixed
+// order and applies the same epilogue.
+//
+// Every mbarrier wait is bounded (clock budget); a wait that runs out sets a
+// shared abort flag and the device status word, the roles drain their own
+// in-flight copies and MMAs, TMEM is freed and the kernel returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace vlaq {
+
+__device__ unsigned int g_vlaq_status = 0;
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 512;
+
+template <bool FP4, int BN>
+struct Cfg {
+  static constexpr int A_BYTES = kBM * 128;
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int NRB = BN / 128;                  // 128-row scale blocks per B tile
+  static constexpr int SFA_BYTES = FP4 ? 4 * 512 : 0;   // 4 k-atoms
+  static constexpr int SFB_BYTES = FP4 ? NRB * 4 * 512 : 0;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGES = (220 * 1024) / STAGE_BYTES > 8 ? 8 : (220 * 1024) / STAGE_BYTES;
+  static constexpr int ACC_BUFS = (BN <= 128) ? 2 : 1;
+  static constexpr int SFA_COL = ACC_BUFS * BN;         // 2 buffers x 16 columns
+  static constexpr int SFB_COL = SFA_COL + 32;          // 2 buffers x NRB*16 columns
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+  static_assert(SFB_COL + 2 * NRB * 16 <= kTmemCols, "TMEM budget");
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+  // Instruction descriptors (M = 128, N = BN, K-major A and B).
+  static constexpr uint32_t IDESC =
+      FP4 ? ((1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBM >> 4) << 24))
+          : ((1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBM >> 4) << 24));
+};
+
+struct GemmArgs {
+  const uint8_t* xs;            // activation tiled scales (NVFP4)
+  const uint8_t* ws;            // weight tiled scales (NVFP4)
+  const float* xg;              // g_x[M] or s_x[M]
+  const float* wg;              // g_w[1] or s_w[N]
+  const __nv_bfloat16* residual;
+  __nv_bfloat16* Y;
+  float* partial;               // [splits][M][N] when splits > 1
+  int M, N, K;
+  int k_steps;                  // MMA k-steps (64 fp4 or 32 fp8 elements each)
+  int k_tiles;                  // stages of 4 k-steps
+  int m_tiles, n_tiles, splits;
+  int units;                    // m_tiles * n_tiles * splits
+  int ka;                       // 512-byte scale atoms per 128-row block = ceil(K/64)
+  int w_row_blocks;             // ceil(N/128)
+  long long budget;             // cycles per bounded wait
+};
+
+struct Unit {
+  int m, n, split, kt0, kt1;
+};
+
+__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
+  Unit r;
+  r.m = u % a.m_tiles;
+  const int t = u / a.m_tiles;
+  r.split = t % a.splits;
+  r.n = t / a.splits;
+  r.kt0 = static_cast<int>(static_cast<long long>(r.split) * a.k_tiles / a.splits);
+  r.kt1 = static_cast<int>(static_cast<long long>(r.split + 1) * a.k_tiles / a.splits);
+  return r;
+}
+
+__device__ __forceinline__ void raise_abort(volatile int* abort_flag) {
+  *abort_flag = 1;
+  atomicOr(&g_vlaq_status, kStatusTimeout);
+}
+
+// Bounded wait that also gives up as soon as another role aborted.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, long long budget,
+                                              volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > budget) {
+      raise_abort(abort_flag);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// fp32 partial sums of one 32-column row segment (split-K).
+__device__ __forceinline__ void store_partial(const GemmArgs& a, int split, int row, int col0,
+                                              const uint32_t (&r)[32]) {
+  float* dst = a.partial + (static_cast<size_t>(split) * a.M + row) * a.N + col0;
+  if (col0 + 32 <= a.N) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      reinterpret_cast<float4*>(dst)[j] =
+          make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                      __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (col0 + j < a.N) dst[j] = __uint_as_float(r[j]);
+  }
+}
+
+// Scale, residual add, bf16 round and store of one 32-column row segment.
+template <bool FP4>
+__device__ __forceinline__ void store_output(const GemmArgs& a, int row, int col0, float rs,
+                                             const uint32_t (&r)[32]) {
+  const bool full = col0 + 32 <= a.N;
+  float y[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float sc = FP4 ? rs : rs * ((col0 + j < a.N) ? a.wg[col0 + j] : 0.0f);
+    y[j] = __uint_as_float(r[j]) * sc;
+  }
+  const size_t base = static_cast<size_t>(row) * a.N + col0;
+  if (a.residual) {
+    if (full) {
+      const uint4* rp = reinterpret_cast<const uint4*>(a.residual + base);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 v = __ldg(rp + j);
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          y[8 * j + 2 * t] += __uint_as_float(wv[t] << 16);
+          y[8 * j + 2 * t + 1] += __uint_as_float(wv[t] & 0xFFFF0000u);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col0 + j < a.N) y[j] += __bfloat162float(a.residual[base + j]);
+    }
+  }
+  if (full) {
+    uint4* yp = reinterpret_cast<uint4*>(a.Y + base);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      yp[j] = make_uint4(pack_bf16x2(y[8 * j], y[8 * j + 1]), pack_bf16x2(y[8 * j + 2], y[8 * j + 3]),
+                         pack_bf16x2(y[8 * j + 4], y[8 * j + 5]), pack_bf16x2(y[8 * j + 6], y[8 * j + 7]));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (col0 + j < a.N) a.Y[base + j] = __float2bfloat16_rn(y[j]);
+  }
+}
+
+template <bool FP4, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+            const GemmArgs args) {
+  using C = Cfg<FP4, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[C::STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
+  __shared__ __align__(8) uint64_t accf_bar[C::ACC_BUFS];
+  __shared__ __align__(8) uint64_t acce_bar[C::ACC_BUFS];
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t s_tmem_base;
+  __shared__ volatile int s_abort;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < C::ACC_BUFS; ++i) {
+      mbar_init(&accf_bar[i], 1);
+      mbar_init(&acce_bar[i], 4);
+    }
+    mbar_init(&drain_bar, 1);
+    s_abort = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&s_tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_phase = 0;  // per-stage bitmask / last armed parity
+      bool ok = true;
+      for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
+        const Unit w = decode_unit(args, u);
+        for (int kt = w.kt0; kt < w.kt1; ++kt) {
+          if (!wait_or_abort(&empty_bar[stage], phase ^ 1u, args.budget, &s_abort)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          uint8_t* sb = sa + C::A_BYTES;
+          const int steps = min(4, args.k_steps - 4 * kt);
+          uint32_t bytes = C::A_BYTES + C::B_BYTES;
+          int nrb = 0;
+          if (FP4) {
+            nrb = min(C::NRB, args.w_row_blocks - w.n * C::NRB);
+            bytes += static_cast<uint32_t>(steps * 512 * (1 + nrb));
+          }
+          mbar_arrive_expect_tx(&full_bar[stage], bytes);
+          armed |= 1u << stage;
+          armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+          tma_load_2d(sa, &tmA, &full_bar[stage], kt * 128, w.m * kBM);
+          tma_load_2d(sb, &tmB, &full_bar[stage], kt * 128, w.n * BN);
+          if (FP4) {
+            uint8_t* ssfa = sb + C::B_BYTES;
+            uint8_t* ssfb = ssfa + C::SFA_BYTES;
+            bulk_load(ssfa, args.xs + (static_cast<size_t>(w.m) * args.ka + 4 * kt) * 512,
+                      steps * 512, &full_bar[stage]);
+            for (int rb = 0; rb < nrb; ++rb)
+              bulk_load(ssfb + rb * 2048,
+                        args.ws + (static_cast<size_t>(w.n * C::NRB + rb) * args.ka + 4 * kt) * 512,
+                        steps * 512, &full_bar[stage]);
+          }
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // drain: let every load this thread issued land before teardown
+        for (int i = 0; i < C::STAGES; ++i)
+          if (armed & (1u << i)) {
+            const long long t0 = clock64();
+            while (!mbar_try_wait(&full_bar[i], (armed_phase >> i) & 1u) &&
+                   clock64() - t0 < args.budget) {
+            }
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      uint32_t sf_buf = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
+        const Unit w = decode_unit(args, u);
+        if (!wait_or_abort(&acce_bar[acc], acc_phase ^ 1u, args.budget, &s_abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * BN);
+        for (int kt = w.kt0; kt < w.kt1; ++kt) {
+          if (!wait_or_abort(&full_bar[stage], phase, args.budget, &s_abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          uint8_t* sb = sa + C::A_BYTES;
+          const int steps = min(4, args.k_steps - 4 * kt);
+          const uint32_t sfa_base = tmem + C::SFA_COL + sf_buf * 16;
+          const uint32_t sfb_base = tmem + C::SFB_COL + sf_buf * (C::NRB * 16);
+          if (FP4) {
+            const uint32_t ssfa = smem_u32(sb + C::B_BYTES);
+            const uint32_t ssfb = ssfa + C::SFA_BYTES;
+            for (int j = 0; j < steps; ++j) {
+              tmem_cp_32x128b_warpx4(sfa_base + 4 * j, sdesc_sf_block(ssfa + 512 * j));
+#pragma unroll
+              for (int rb = 0; rb < C::NRB; ++rb)
+                tmem_cp_32x128b_warpx4(sfb_base + C::NRB * 4 * j + 4 * rb,
+                                       sdesc_sf_block(ssfb + rb * 2048 + 512 * j));
+            }
+          }
+          const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
+          for (int j = 0; j < steps; ++j) {
+            const uint64_t ad = sdesc_kmajor_sw128(a0 + 32 * j);
+            const uint64_t bd = sdesc_kmajor_sw128(b0 + 32 * j);
+            const uint32_t accum = (kt > w.kt0 || j > 0) ? 1u : 0u;
+            if (FP4)
+              mma_mxf4nvf4(d_tmem, ad, bd, C::IDESC, sfa_base + 4 * j, sfb_base + C::NRB * 4 * j,
+                           accum);
+            else
+              mma_f8f6f4(d_tmem, ad, bd, C::IDESC, accum);
+          }
+          umma_commit(&empty_bar[stage]);
+          sf_buf ^= 1u;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&accf_bar[acc]);
+        if (++acc == C::ACC_BUFS) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      // drain: every tcgen05 op issued by this thread completes before TMEM
+      // is released
+      umma_commit(&drain_bar);
+      const long long t0 = clock64();
+      while (!mbar_try_wait(&drain_bar, 0) && clock64() - t0 < 4 * args.budget + 1000000) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM sub-partition this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
+      const Unit w = decode_unit(args, u);
+      if (!wait_or_abort(&accf_bar[acc], acc_phase, args.budget, &s_abort)) break;
+      tc_fence_after();
+      const int row = w.m * kBM + 32 * q + lane;
+      const bool row_ok = row < args.M;
+      float rs = 0.0f;
+      if (row_ok && args.splits == 1) rs = FP4 ? args.xg[row] * args.wg[0] : args.xg[row];
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        __syncwarp();
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tbase + c0, r);
+        tmem_ld_wait();
+        const int col0 = w.n * BN + c0;
+        if (row_ok && col0 < args.N) {
+          if (args.splits > 1)
+            store_partial(args, w.split, row, col0, r);
+          else
+            store_output<FP4>(args, row, col0, rs, r);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce_bar[acc]);
+      if (++acc == C::ACC_BUFS) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Split-K reduction + epilogue: fixed split order, same scaling as the
+// direct epilogue.  8 outputs per thread.
+template <bool FP4>
+__global__ void splitk_reduce_kernel(const float* __restrict__ partial, int splits, int M, int N,
+                                     const float* __restrict__ xg, const float* __restrict__ wg,
+                                     const __nv_bfloat16* __restrict__ residual,
+                                     __nv_bfloat16* __restrict__ Y) {
+  const int64_t idx8 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t total8 = static_cast<int64_t>(M) * N / 8;
+  if (idx8 >= total8) return;
+  const int64_t e0 = idx8 * 8;
+  const int row = static_cast<int>(e0 / N);
+  const int col = static_cast<int>(e0 % N);
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+  for (int s = 0; s < splits; ++s) {
+    const float4* p = reinterpret_cast<const float4*>(partial + (static_cast<size_t>(s) * M) * N + e0);
+    const float4 a = p[0], b = p[1];
+    acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+    acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+  }
+  const float rs = FP4 ? xg[row] * wg[0] : xg[row];
+  float y[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) y[j] = acc[j] * (FP4 ? rs : rs * wg[col + j]);
+  if (residual) {
+    const uint4 v = *reinterpret_cast<const uint4*>(residual + e0);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      y[2 * t] += __uint_as_float(wv[t] << 16);
+      y[2 * t + 1] += __uint_as_float(wv[t] & 0xFFFF0000u);
+    }
+  }
+  *reinterpret_cast<uint4*>(Y + e0) = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
+                                                 pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+}
+
+// ------------------------------------------------------------ host side --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D byte tensor [rows, row_bytes] with the given pitch, box 128 x box_rows,
+// 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows, uint64_t pitch,
+              uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {pitch};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool FP4, int BN>
+cudaError_t run(const uint8_t* xq, const uint8_t* xs, const float* xg, const uint8_t* wq, const uint8_t* ws,
+                const float* wg, const void* residual, void* Y, int64_t M, int64_t N, int64_t K,
+                void* workspace, const GemmPlan& plan, long long budget, cudaStream_t s) {
+  using C = Cfg<FP4, BN>;
+  const int64_t pitch = FP4 ? nvfp4_code_pitch(K) : K;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, xq, static_cast<uint64_t>(pitch), static_cast<uint64_t>(M), static_cast<uint64_t>(pitch), kBM) ||
+      !make_map(&tb, wq, static_cast<uint64_t>(pitch), static_cast<uint64_t>(N), static_cast<uint64_t>(pitch), BN))
+    return cudaErrorInvalidValue;
+  GemmArgs a;
+  a.xs = xs;
+  a.ws = ws;
+  a.xg = xg;
+  a.wg = wg;
+  a.residual = static_cast<const __nv_bfloat16*>(residual);
+  a.Y = static_cast<__nv_bfloat16*>(Y);
+  a.partial = static_cast<float*>(workspace);
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.k_steps = static_cast<int>(FP4 ? (K + 63) / 64 : (K + 31) / 32);
+  a.k_tiles = (a.k_steps + 3) / 4;
+  a.m_tiles = static_cast<int>((M + kBM - 1) / kBM);
+  a.n_tiles = static_cast<int>((N + BN - 1) / BN);
+  a.splits = plan.splits;
+  a.units = a.m_tiles * a.n_tiles * a.splits;
+  a.ka = static_cast<int>((K + 63) / 64);
+  a.w_row_blocks = static_cast<int>((N + 127) / 128);
+  a.budget = budget;
+  auto kern = gemm_kernel<FP4, BN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int grid = plan.grid < a.units ? plan.grid : a.units;
+  kern<<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || plan.splits == 1) return e;
+  const int64_t total8 = M * N / 8;
+  const int threads = 256;
+  const int64_t blocks = (total8 + threads - 1) / threads;
+  splitk_reduce_kernel<FP4><<<static_cast<unsigned int>(blocks), threads, 0, s>>>(
+      static_cast<const float*>(workspace), plan.splits, a.M, a.N, xg, wg,
+      static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(Y));
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+GemmPlan plan_gemm(bool fp4, int64_t M, int64_t N, int64_t K, int num_sms) {
+  GemmPlan p;
+  p.bn = 128;
+  const int64_t k_steps = fp4 ? (K + 63) / 64 : (K + 31) / 32;
+  const int64_t k_tiles = (k_steps + 3) / 4;
+  const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + p.bn - 1) / p.bn);
+  int64_t splits = 1;
+  if (tiles * 2 <= num_sms) {
+    splits = num_sms / tiles;
+    if (splits > k_tiles / 2) splits = k_tiles / 2;
+    if (splits < 1) splits = 1;
+  }
+  p.splits = static_cast<int>(splits);
+  const int64_t units = tiles * splits;
+  p.grid = static_cast<int>(units < num_sms ? units : num_sms);
+  p.ws_bytes = splits > 1 ? static_cast<size_t>(splits) * M * N * sizeof(float) : 0;
+  return p;
+}
+
+cudaError_t launch_linear(bool fp4, const uint8_t* xq, const uint8_t* xs, const float* xg, const uint8_t* wq,
+                          const uint8_t* ws, const float* wg, const void* residual, void* Y, int64_t M, int64_t N,
+                          int64_t K, void* workspace, size_t ws_bytes, const GemmPlan& plan, long long budget,
+                          cudaStream_t s) {
+  (void)ws_bytes;
+  if (fp4) return run<true, 128>(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
+  return run<false, 128>(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
+}
+
+cudaError_t read_and_clear_status(unsigned int* out, cudaStream_t s) {
+  cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_vlaq_status, sizeof(unsigned int), 0,
+                                            cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return e;
+  const unsigned int zero = 0;
+  e = cudaMemcpyToSymbolAsync(g_vlaq_status, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return e;
+  return cudaStreamSynchronize(s);
+}
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  static int cache[64] = {0};
+  if (dev < 64 && cache[dev]) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev < 64) cache[dev] = n;
+  return n;
+}
+
+}  // namespace vlaq

@@ -1,0 +1,54 @@
+// Internal launcher interface between the C-ABI layer (api.cu) and the
+// kernels (quant.cu, gemm.cu).  Arguments are validated by the caller.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace vlaq {
+
+// Device status word bits (read and cleared by vlaq_check).
+enum : unsigned int { kStatusTimeout = 1u };
+
+// Largest K the one-thread-per-64-block prologue supports (512 threads).
+constexpr int64_t kMaxQuantK = 32768;
+
+constexpr uint32_t kFlagRmsNorm = 1u;
+constexpr uint32_t kFlagHadamard = 2u;
+
+inline int64_t nvfp4_code_pitch(int64_t K) { return (K + 63) / 64 * 32; }
+inline int64_t nvfp4_scale_cols_padded(int64_t K) { return (K + 63) / 64 * 4; }
+inline int64_t nvfp4_rows_padded(int64_t rows) { return (rows + 127) / 128 * 128; }
+
+// ---- prologue / quantizer kernels (quant.cu)
+cudaError_t launch_quant_act_nvfp4(const void* X, int64_t M, int64_t K, const void* gamma, float eps,
+                                   uint32_t flags, uint8_t* codes, uint8_t* scales, float* g_x,
+                                   cudaStream_t s);
+cudaError_t launch_quant_weight_nvfp4(const void* W, int64_t N, int64_t K, uint32_t flags,
+                                      uint8_t* codes, uint8_t* scales, float* g_w, cudaStream_t s);
+cudaError_t launch_quant_fp8(const void* X, int64_t rows, int64_t K, const void* gamma, float eps,
+                             uint32_t flags, uint8_t* codes, float* s_out, cudaStream_t s);
+
+// ---- GEMM (gemm.cu)
+struct GemmPlan {
+  int bn;          // tile width along N
+  int splits;      // split-K factor (1 = direct epilogue)
+  int grid;        // persistent CTAs
+  size_t ws_bytes; // fp32 partials needed when splits > 1
+};
+GemmPlan plan_gemm(bool fp4, int64_t M, int64_t N, int64_t K, int num_sms);
+
+cudaError_t launch_linear(bool fp4, const uint8_t* xq, const uint8_t* xs, const float* xg,
+                          const uint8_t* wq, const uint8_t* ws, const float* wg,
+                          const void* residual, void* Y, int64_t M, int64_t N, int64_t K,
+                          void* workspace, size_t ws_bytes, const GemmPlan& plan,
+                          long long wait_budget, cudaStream_t s);
+
+// Device status word accessors (gemm.cu).
+cudaError_t read_and_clear_status(unsigned int* out, cudaStream_t s);
+
+// Current device's SM count (cached per device).
+int device_sm_count();
+
+}  // namespace vlaq
