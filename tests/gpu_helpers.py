@@ -12,8 +12,8 @@ REL_FRO_TOL = 2e-3  # GEMM gate: relative Frobenius error vs the fp64 oracle
 
 def vq():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device (no fallback exists)"
-    from vlaq_quantize_act_b200 import build
-    build.build()
+    from conftest import build_library
+    build_library()
     import vlaq_quantize_act_b200 as m
     return m
 

@@ -14,8 +14,8 @@ GOLDEN = os.path.join(ROOT, "tests", "golden", "k3420_rejection.txt")
 
 @pytest.fixture(scope="module")
 def vq():
-    from vlaq_quantize_act_b200 import build
-    build.build()
+    from conftest import build_library
+    build_library()
     import vlaq_quantize_act_b200 as vq
     return vq
 

@@ -1,6 +1,6 @@
 """Builds the CUDA library libvlaq.so in-tree (sm_100a only).
 
-    python -m vlaq_quantize_act_b200.build [--force]
+    python vlaq_quantize_act_b200/build.py [--force]
 
 nvcc compiles every .cu under csrc/ with -gencode arch=compute_100a,code=sm_100a
 and links them into vlaq_quantize_act_b200/libvlaq.so with the CUDA runtime
