@@ -174,6 +174,27 @@ VLAQ_API vlaq_status vlaq_linear_nvfp4(const uint8_t* xq, const uint8_t* xs,
                               int64_t N, int64_t K, void* workspace,
                               size_t ws_bytes, void* stream);
 
+/* Same computation, arguments and rules as vlaq_linear_nvfp4, for callers
+ * that cannot allocate device memory (a host callback, a real-time control
+ * loop that must not touch the allocator, an embedding whose arena owns all
+ * device memory): no workspace argument, and the call never allocates.
+ * The split-K partial sums of small-M shapes go to a 4 MiB array compiled
+ * into the library, which every GPU that loads the library holds until the
+ * process exits.  A shape whose split-K plan needs more than 4 MiB is refused
+ * with VLAQ_ERR_WORKSPACE (use vlaq_linear_nvfp4 then).  The first call on
+ * each device looks the array's address up (cudaGetSymbolAddress) and caches
+ * it; make that first call before any stream capture.  All calls on a
+ * device share the array and it keeps the last call's contents (nothing in
+ * it has to start at zero: every partial is written before it is read);
+ * calls that overlap on the GPU, e.g. on two streams, race on it and must
+ * be serialized by the caller.  The source pages have no counterpart of
+ * this entry point. */
+VLAQ_API vlaq_status vlaq_linear_nvfp4_noalloc(const uint8_t* xq, const uint8_t* xs,
+                                      const float* g_x, const uint8_t* wq,
+                                      const uint8_t* ws, const float* g_w,
+                                      const void* residual, void* Y, int64_t M,
+                                      int64_t N, int64_t K, void* stream);
+
 /* ------------------------------------------------------------ FP8 W8A8 */
 
 /* Per-row weight quantization: s_w[n] = max|w_n| / 448, codes E4M3.

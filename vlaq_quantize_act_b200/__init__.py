@@ -21,7 +21,7 @@ __all__ = [
     "vlaq_last_error", "vlaq_version", "vlaq_check",
     "vlaq_nvfp4_code_pitch", "vlaq_nvfp4_scale_bytes", "vlaq_linear_workspace_bytes",
     "vlaq_quantize_weight_nvfp4", "vlaq_quantize_act_nvfp4", "vlaq_linear_nvfp4",
-    "vlaq_quantize_weight_fp8", "vlaq_quantize_act_fp8", "vlaq_linear_fp8",
+    "vlaq_quantize_weight_fp8", "vlaq_quantize_act_fp8", "vlaq_linear_fp8", "vlaq_linear_nvfp4_noalloc",
     "alloc_nvfp4", "alloc_fp8", "alloc_workspace",
 ]
 
@@ -59,6 +59,7 @@ _SIGS = {
     "vlaq_quantize_weight_fp8": (ctypes.c_int, [_P, _I64, _I64, _U32, _P, _P, _P]),
     "vlaq_quantize_act_fp8": (ctypes.c_int, [_P, _I64, _I64, _P, _F, _U32, _P, _P, _P]),
     "vlaq_linear_fp8": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
+    "vlaq_linear_nvfp4_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -134,6 +135,13 @@ def vlaq_linear_nvfp4(xq, xs, g_x, wq, ws, g_w, residual, Y, M, N, K, workspace=
                       stream=None):
     _check(_lib.vlaq_linear_nvfp4(_ptr(xq), _ptr(xs), _ptr(g_x), _ptr(wq), _ptr(ws), _ptr(g_w), _ptr(residual),
                                   _ptr(Y), M, N, K, _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def vlaq_linear_nvfp4_noalloc(xq, xs, g_x, wq, ws, g_w, residual, Y, M, N, K, stream=None):
+    """vlaq_linear_nvfp4 for callers that cannot allocate: no workspace; the
+    split-K scratch is a fixed 4 MiB array inside the library (see vlaq.h)."""
+    _check(_lib.vlaq_linear_nvfp4_noalloc(_ptr(xq), _ptr(xs), _ptr(g_x), _ptr(wq), _ptr(ws), _ptr(g_w),
+                                          _ptr(residual), _ptr(Y), M, N, K, _stream(stream)))
 
 
 # ------------------------------------------------------------------- FP8

@@ -255,4 +255,29 @@ vlaq_status vlaq_linear_fp8(const uint8_t* xq, const float* s_x, const uint8_t* 
                        ws_bytes, stream);
 }
 
+vlaq_status vlaq_linear_nvfp4_noalloc(const uint8_t* xq, const uint8_t* xs, const float* g_x, const uint8_t* wq,
+                                      const uint8_t* ws, const float* g_w, const void* residual, void* Y, int64_t M,
+                                      int64_t N, int64_t K, void* stream) {
+  const char* fn = "vlaq_linear_nvfp4_noalloc";
+  // Shapes the regular validation accepts get their scratch need checked
+  // against the fixed array; everything else is refused by linear_common
+  // with the usual messages.
+  if (M > 0 && N > 0 && N % 8 == 0 && K > 0 && K % 16 == 0 && M <= 0x7FFFFFFF && N <= 0x7FFFFFFF &&
+      K <= 0x7FFFFFFF) {
+    const size_t need = vlaq::plan_gemm(true, M, N, K, vlaq::device_sm_count()).ws_bytes;
+    if (need > vlaq::kNoallocScratchBytes)
+      return fail(VLAQ_ERR_WORKSPACE,
+                  "%s: shape %lld x %lld x %lld needs %zu bytes of split-K scratch, more than the %zu-byte static "
+                  "scratch array; use vlaq_linear_nvfp4 with a caller-allocated workspace",
+                  fn, (long long)M, (long long)N, (long long)K, need, vlaq::kNoallocScratchBytes);
+  }
+  void* scratch = nullptr;
+  if (M > 0) {
+    cudaError_t e = vlaq::noalloc_scratch(&scratch);
+    if (e != cudaSuccess) return cuda_fail(fn, e);
+  }
+  return linear_common(fn, true, xq, xs, g_x, wq, ws, g_w, residual, Y, M, N, K, scratch,
+                       vlaq::kNoallocScratchBytes, stream);
+}
+
 }  // extern "C"

@@ -51,4 +51,9 @@ cudaError_t read_and_clear_status(unsigned int* out, cudaStream_t s);
 // Current device's SM count (cached per device).
 int device_sm_count();
 
+// ---- static scratch for the allocation-free linear entry point (noalloc.cu)
+constexpr size_t kNoallocScratchBytes = size_t(4) << 20;  // 4 MiB per device
+constexpr int kMaxDevices = 64;
+cudaError_t noalloc_scratch(void** out);
+
 }  // namespace vlaq
