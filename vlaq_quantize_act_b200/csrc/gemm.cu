@@ -40,7 +40,6 @@ __device__ unsigned int g_vlaq_status = 0;
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
 
 template <bool FP4, int BN>
@@ -56,6 +55,9 @@ struct Cfg {
   static constexpr int SFA_COL = ACC_BUFS * BN;         // 2 buffers x 16 columns
   static constexpr int SFB_COL = SFA_COL + 32;          // 2 buffers x NRB*16 columns
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+  // one epilogue warp per (TMEM sub-partition, 128-column half)
+  static constexpr int EPI_WARPS = 4 * NRB;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static_assert(SFB_COL + 2 * NRB * 16 <= kTmemCols, "TMEM budget");
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
   // Instruction descriptors (M = 128, N = BN, K-major A and B).
@@ -184,7 +186,7 @@ __device__ __forceinline__ void store_output(const GemmArgs& a, int row, int col
 }
 
 template <bool FP4, int BN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<FP4, BN>::THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const GemmArgs args) {
   using C = Cfg<FP4, BN>;
@@ -208,7 +210,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     }
     for (int i = 0; i < C::ACC_BUFS; ++i) {
       mbar_init(&accf_bar[i], 1);
-      mbar_init(&acce_bar[i], 4);
+      mbar_init(&acce_bar[i], C::EPI_WARPS);
     }
     mbar_init(&drain_bar, 1);
     s_abort = 0;
@@ -355,7 +357,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM sub-partition this warp may access
+    // Warp e handles TMEM sub-partition (warp % 4) and columns
+    // [128 h, 128 h + 128), h = e / 4.  It copies its 128 accumulator
+    // columns to registers, hands the TMEM buffer back to the MMA issuer at
+    // once, then scales, adds the residual and stores while the next tile's
+    // MMAs run.
+    const int e = warp - 2;
+    const int q = warp & 3;
+    const int h = e >> 2;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
@@ -364,29 +373,31 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       tc_fence_after();
       const int row = w.m * kBM + 32 * q + lane;
       const bool row_ok = row < args.M;
-      float rs = 0.0f;
-      if (row_ok && args.splits == 1) rs = FP4 ? args.xg[row] * args.wg[0] : args.xg[row];
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * BN);
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        __syncwarp();
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tbase + c0, r);
-        tmem_ld_wait();
-        const int col0 = w.n * BN + c0;
-        if (row_ok && col0 < args.N) {
-          if (args.splits > 1)
-            store_partial(args, w.split, row, col0, r);
-          else
-            store_output<FP4>(args, row, col0, rs, r);
-        }
-      }
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16) +
+                             static_cast<uint32_t>(acc * BN + 128 * h);
+      __syncwarp();
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tbase + 32 * c, r[c]);
+      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acce_bar[acc]);
       if (++acc == C::ACC_BUFS) {
         acc = 0;
         acc_phase ^= 1u;
+      }
+      float rs = 0.0f;
+      if (row_ok && args.splits == 1) rs = FP4 ? args.xg[row] * args.wg[0] : args.xg[row];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int col0 = w.n * BN + 128 * h + 32 * c;
+        if (row_ok && col0 < args.N) {
+          if (args.splits > 1)
+            store_partial(args, w.split, row, col0, r[c]);
+          else
+            store_output<FP4>(args, row, col0, rs, r[c]);
+        }
       }
     }
   }
@@ -506,7 +517,7 @@ cudaError_t run(const uint8_t* xq, const uint8_t* xs, const float* xg, const uin
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = plan.grid < a.units ? plan.grid : a.units;
-  kern<<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, a);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, a);
   e = cudaGetLastError();
   if (e != cudaSuccess || plan.splits == 1) return e;
   const int64_t total8 = M * N / 8;
@@ -522,10 +533,22 @@ cudaError_t run(const uint8_t* xq, const uint8_t* xs, const float* xg, const uin
 
 GemmPlan plan_gemm(bool fp4, int64_t M, int64_t N, int64_t K, int num_sms) {
   GemmPlan p;
-  p.bn = 128;
   const int64_t k_steps = fp4 ? (K + 63) / 64 : (K + 31) / 32;
   const int64_t k_tiles = (k_steps + 3) / 4;
-  const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + p.bn - 1) / p.bn);
+  const int64_t m_tiles = (M + kBM - 1) / kBM;
+  // Wide tiles halve the scale-factor copies per FLOP and the A re-reads;
+  // they are used whenever they still give every SM work.
+  const int64_t tiles256 = m_tiles * ((N + 255) / 256);
+  if (tiles256 * 2 > num_sms) {
+    p.bn = 256;
+    p.splits = 1;
+    p.grid = static_cast<int>(tiles256 < num_sms ? tiles256 : num_sms);
+    p.ws_bytes = 0;
+    return p;
+  }
+  // Few output tiles (decode): narrow tiles and split-K over the SMs.
+  p.bn = 128;
+  const int64_t tiles = m_tiles * ((N + 127) / 128);
   int64_t splits = 1;
   if (tiles * 2 <= num_sms) {
     splits = num_sms / tiles;
@@ -544,6 +567,10 @@ cudaError_t launch_linear(bool fp4, const uint8_t* xq, const uint8_t* xs, const 
                           int64_t K, void* workspace, size_t ws_bytes, const GemmPlan& plan, long long budget,
                           cudaStream_t s) {
   (void)ws_bytes;
+  if (plan.bn == 256) {
+    if (fp4) return run<true, 256>(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
+    return run<false, 256>(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
+  }
   if (fp4) return run<true, 128>(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
   return run<false, 128>(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
 }
