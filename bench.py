@@ -262,16 +262,107 @@ def time_graph(g, reps, dist_on, device):
     return max_over_ranks(e0.elapsed_time(e1) / reps, dist_on, device)
 
 
-def kernel_durations(step, reps):
+class _Rt:
+    """CUDA runtime calls for timing events that live inside a graph: an
+    event recorded with cudaEventRecordExternal during stream capture
+    becomes an event-record node that timestamps every replay (a plain
+    record would only become a dependency edge)."""
+    lib = None
+
+    @classmethod
+    def get(cls):
+        if cls.lib is None:
+            import ctypes
+            for name in ("libcudart.so.12", "libcudart.so"):
+                try:
+                    lib = ctypes.CDLL(name)
+                    break
+                except OSError:
+                    lib = None
+            if lib is None:
+                raise OSError("CUDA runtime library not found")
+            P = ctypes.c_void_p
+            lib.cudaEventCreate.argtypes = [ctypes.POINTER(P)]
+            lib.cudaEventRecordWithFlags.argtypes = [P, P, ctypes.c_uint]
+            lib.cudaEventElapsedTime.argtypes = [ctypes.POINTER(ctypes.c_float), P, P]
+            lib.cudaEventDestroy.argtypes = [P]
+            cls.lib = lib
+        return cls.lib
+
+
+class GraphEvent:
+    def __init__(self):
+        import ctypes
+        self.h = ctypes.c_void_p()
+        rc = _Rt.get().cudaEventCreate(ctypes.byref(self.h))
+        if rc != 0:
+            raise RuntimeError(f"cudaEventCreate failed ({rc})")
+
+    def record(self):
+        rc = _Rt.get().cudaEventRecordWithFlags(self.h, ctypes_stream(), 1)  # cudaEventRecordExternal
+        if rc != 0:
+            raise RuntimeError(f"cudaEventRecordWithFlags failed ({rc})")
+
+    def elapsed_time(self, other):
+        import ctypes
+        ms = ctypes.c_float()
+        rc = _Rt.get().cudaEventElapsedTime(ctypes.byref(ms), self.h, other.h)
+        if rc != 0:
+            raise RuntimeError(f"cudaEventElapsedTime failed ({rc})")
+        return ms.value
+
+
+def ctypes_stream():
+    import ctypes
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def kernel_durations(step, reps, copies=1):
     """Per-launch durations (ms) of the prologue and the GEMM of each
-    projection, CUDA events on the launching stream."""
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in step.layers] for _ in range(reps)]
-    for r in range(reps):
-        step.run(r, evs[r])
-    torch.cuda.synchronize()
-    pro = [[evs[r][i][0].elapsed_time(evs[r][i][1]) for r in range(reps)] for i in range(len(step.layers))]
-    gem = [[evs[r][i][1].elapsed_time(evs[r][i][2]) for r in range(reps)] for i in range(len(step.layers))]
-    return pro, gem
+    projection from CUDA events on the launching stream, recorded as event
+    nodes inside a CUDA graph of the step (host launch overhead cannot leak
+    into the kernel times).  Falls back to eager event pairs if the runtime
+    refuses.  Returns (prologue[i][r], gemm[i][r], mode)."""
+    pro = [[] for _ in step.layers]
+    gem = [[] for _ in step.layers]
+
+    def collect(evs):
+        for c in range(copies):
+            for i in range(len(step.layers)):
+                pro[i].append(evs[c][i][0].elapsed_time(evs[c][i][1]))
+                gem[i].append(evs[c][i][1].elapsed_time(evs[c][i][2]))
+
+    try:
+        evs = [[[GraphEvent() for _ in range(3)] for _ in step.layers] for _ in range(copies)]
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for c in range(copies):
+                step.run(c, evs[c])
+        torch.cuda.synchronize()
+        for _ in range(2):
+            g.replay()
+        torch.cuda.synchronize()
+        for _ in range(reps):
+            g.replay()
+            torch.cuda.synchronize()
+            collect(evs)
+        del g
+        return pro, gem, "graph"
+    except Exception as exc:  # noqa: BLE001
+        torch.cuda.synchronize()
+        print(f"bench: in-graph event timing unavailable ({exc}); using eager events", file=sys.stderr)
+        pro = [[] for _ in step.layers]
+        gem = [[] for _ in step.layers]
+        for _ in range(reps):
+            evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in step.layers]
+                   for _ in range(copies)]
+            for c in range(copies):
+                step.run(c, evs[c])
+            torch.cuda.synchronize()
+            collect(evs)
+        return pro, gem, "eager"
 
 
 # -------------------------------------------------------------- CPU oracle
@@ -373,7 +464,7 @@ def main():
     sampler.start()
     time.sleep(0.3)
     ms = time_graph(graph, args.steps, dist_on, device)
-    pro, gem = kernel_durations(step, max(args.steps // 2, 3))
+    pro, gem, tmode = kernel_durations(step, max(args.steps // 2, 3))
     clocks = sampler.stop()
     value = world * step.flops / (ms / 1e3) / 1e12
     # dominant kernel: the gate_up GEMM launch (about half of the step)
@@ -404,7 +495,7 @@ def main():
         "roofline": {"bound": "tensor", "achieved": g_ach, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": g_ach / fp4_peak, "traffic": traffic,
                      "kernel": "gemm_kernel<FP4> gate_up 1024x37888x3584 (2MNK = 278.1 GFLOP per launch)",
-                     "all_gemms_tflops": gemm_all,
+                     "all_gemms_tflops": gemm_all, "timing": f"CUDA events in a {tmode} capture of the step",
                      "peak_note": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 4 (nominal FP4:BF16)"},
         "prologue": {"bound": "hbm", "achieved": p_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": p_ach / peaks["hbm_gbs"], "kernel": "quant_rows_kernel<NVFP4>"},
@@ -421,7 +512,7 @@ def main():
             dgraph.replay()
         dms = time_graph(dgraph, args.steps, dist_on, device) / 2
         dbytes = sum(dstep.gemm_bytes(L) + dstep.prologue_bytes(L) for L in dstep.layers)
-        dpro, dgem = kernel_durations(dstep, max(args.steps // 2, 4))
+        dpro, dgem, _ = kernel_durations(dstep, max(args.steps // 2, 4), copies=2)
         dgem_ms = sum(sum(x) for x in dgem) / len(dgem[0])
         dgem_bytes = sum(dstep.gemm_bytes(L) for L in dstep.layers)
         out["decode"] = {"value": world * dbytes / (dms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": dms,
@@ -439,7 +530,7 @@ def main():
         for _ in range(args.warmup):
             fgraph.replay()
         fms = time_graph(fgraph, args.steps, dist_on, device)
-        _, fgem = kernel_durations(fstep, max(args.steps // 2, 3))
+        _, fgem, _ = kernel_durations(fstep, max(args.steps // 2, 3))
         fgem_ms = sum(sum(x) for x in fgem) / len(fgem[0])
         fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
         out["fp8"] = {"value": world * fstep.flops / (fms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": fms,

@@ -99,3 +99,44 @@ def test_weight_fp8(N, K, flags):
     gc, gs = gpu_quant_fp8(W, flags=flags, weight=True)
     assert np.array_equal(gc, rc)
     assert np.array_equal(gs.view(np.uint32), rs.view(np.uint32))
+
+
+@pytest.mark.parametrize("flags", [0, 2, 3])
+def test_act_nvfp4_stress_many_quotients(flags):
+    """8M quotients (fp32-valued after the rotation): every code and scale
+    bit-exact; exercises the reciprocal shortcut and its exact fallback."""
+    M, K = 2048, 4096
+    X = _inputs(M, K, 77 + flags)
+    gam = si.norm_gain(K, 77)
+    ref = oracle.quantize_nvfp4(bits(X), bits(gam), 1e-6, flags)
+    assert_nvfp4_equal(gpu_quant_act_nvfp4(X, gam, 1e-6, flags), ref, M, K, f"stress f{flags}")
+
+
+@pytest.mark.parametrize("flags", [0, 2])
+def test_act_fp8_stress_many_quotients(flags):
+    M, K = 1024, 4096
+    X = _inputs(M, K, 88 + flags)
+    rc, rs = oracle.quantize_fp8(bits(X), flags=flags)
+    gc, gs = gpu_quant_fp8(X, flags=flags)
+    assert np.array_equal(gc, rc), f"{int((gc != rc).sum())} fp8 codes differ"
+    assert np.array_equal(gs.view(np.uint32), rs.view(np.uint32))
+
+
+def test_act_nvfp4_values_near_decision_points():
+    """Rows whose quotients sit on and next to every E2M1 decision point:
+    amax 6 makes the block scale ~1, elements are midpoints scaled by
+    1 + k/256 (bf16-representable neighbours)."""
+    rows = []
+    mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    for j in range(-8, 9):
+        r = np.zeros(64, np.float32)
+        r[0] = 6.0
+        for i, m in enumerate(mids):
+            r[1 + i] = m * (1 + j / 256.0)
+            r[9 + i] = -m * (1 - j / 256.0)
+        rows.append(r)
+    X = torch.from_numpy(np.stack(rows)).to(torch.bfloat16)
+    for scale in (1.0, 2.0 ** -20, 2.0 ** 20, 3.0, 0.1):
+        Xs = (X.float() * scale).to(torch.bfloat16)
+        ref = oracle.quantize_nvfp4(bits(Xs))
+        assert_nvfp4_equal(gpu_quant_act_nvfp4(Xs), ref, Xs.shape[0], 64, f"near points x{scale}")
