@@ -130,3 +130,36 @@ def test_workspace_is_checked():
     with pytest.raises(m.VlaqError) as ei:
         m.vlaq_linear_nvfp4(xq, xs, xg, wq, ws, wg, None, Y, M, N, K, None, 0)
     assert ei.value.status == 7
+
+
+# Shapes with more than 74 output tiles of 128 x 256 take the wide-tile
+# prefill kernel (scale writers + early TMEM release); ragged M, N and K.
+WIDE_CASES = [
+    (1024, 2560, 1024, False),
+    (1000, 2568, 336, True),
+    (777, 4096, 512, True),
+]
+
+
+@pytest.mark.parametrize("M,N,K,res", WIDE_CASES)
+def test_linear_nvfp4_wide_tiles_vs_oracle(M, N, K, res):
+    m = vq()
+    assert m.vlaq_linear_workspace_bytes(M, N, K) == 0
+    case = _oracle_case(M, N, K, 23, residual=res)
+    Y = _run_nvfp4_from_oracle(M, N, K, case)
+    rel, mx = gemm_error(Y, case[-1])
+    print(f"nvfp4 wide M={M} N={N} K={K} res={res}: rel_fro={rel:.3e} max_abs={mx:.3e}")
+    assert rel < REL_FRO_TOL, (rel, mx)
+
+
+@pytest.mark.parametrize("M,N,K,res", WIDE_CASES[:2])
+def test_linear_fp8_wide_tiles_vs_oracle(M, N, K, res):
+    X = si.projection_activations(K, M, 33)
+    W = si.projection_weight(K, N, 33)
+    cx, sx = oracle.quantize_fp8(bits(X))
+    cw, sw = oracle.quantize_fp8(bits(W))
+    R = si.residual(M, N, 33) if res else None
+    Y64 = oracle.linear_f64(oracle.decode_fp8(cx, sx), oracle.decode_fp8(cw, sw), None if R is None else bits(R))
+    Y = gpu_linear_fp8(to_dev(cx), to_dev(sx), to_dev(cw), to_dev(sw), M, N, K, None if R is None else R.cuda())
+    rel, mx = gemm_error(Y, Y64)
+    assert rel < REL_FRO_TOL, (rel, mx)

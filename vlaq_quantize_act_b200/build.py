@@ -22,6 +22,28 @@ FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std
          "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr"]
 
 
+# Kernels that re-split registers between warpgroups with setmaxnreg: the
+# per-warpgroup budgets they request add up to exactly this entry register
+# count times the block size, so ptxas must allocate exactly this many at
+# entry (fewer would make setmaxnreg.inc wait for registers that never free).
+ENTRY_REGISTERS = {"gemm_fp4_sfw_kernel": 128}
+
+
+def _check_entry_registers(ptxas_log: str) -> None:
+    current = None
+    for line in ptxas_log.splitlines():
+        if "Compiling entry function" in line:
+            current = line
+        elif current and "Used" in line and "registers" in line:
+            for name, regs in ENTRY_REGISTERS.items():
+                if name in current:
+                    used = int(line.split("Used")[1].split("registers")[0])
+                    if used != regs:
+                        raise RuntimeError(f"{name}: ptxas allocated {used} registers at entry, "
+                                           f"the setmaxnreg split needs exactly {regs}")
+            current = None
+
+
 def _sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
@@ -46,10 +68,13 @@ def build(force: bool = False, verbose: bool = False) -> str:
     objs = []
     for src in _sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [NVCC, *FLAGS, "-c", src, "-o", obj]
-        if verbose:
-            cmd.insert(1, "-Xptxas=-v")
-        subprocess.run(cmd, check=True)
+        cmd = [NVCC, *FLAGS, "-Xptxas=-v", "-c", src, "-o", obj]
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        if verbose or res.returncode != 0:
+            sys.stderr.write(res.stdout + res.stderr)
+        if res.returncode != 0:
+            raise subprocess.CalledProcessError(res.returncode, cmd)
+        _check_entry_registers(res.stderr)
         objs.append(obj)
     tmp = OUT + ".tmp"
     subprocess.run([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs, "-o", tmp,

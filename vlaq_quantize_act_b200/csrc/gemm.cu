@@ -411,6 +411,274 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   }
 }
 
+// ----------------------------------------------------------------------------
+// NVFP4 GEMM with dedicated scale-factor writers (prefill shapes, BN = 256).
+//
+// The block scales reach TMEM through registers (tcgen05.st) from four
+// "scale writer" warps, one per TMEM sub-partition, into NSF rotating TMEM
+// buffers, instead of tcgen05.cp issued by the MMA thread: the single MMA
+// issuer then only waits, issues four MMAs per stage and commits.  Layout of
+// one scale buffer is the one the block-scaled MMA reads (per k-step, 4
+// columns of A scales and 8 of B scales; lane r0 + 32 q of column c holds
+// the four block scales of row r0 + 32 c, replicated in every q).
+//   warps 0-3   (warpgroup 0): TMA producer (warp 0), TMEM allocator + MMA
+//               issuer (warp 1), warps 2-3 idle;
+//   warps 4-11  (warpgroups 1, 2): epilogue, registers raised to 168;
+//   warps 12-15 (warpgroup 3): scale writers, registers lowered to 48.
+// The warpgroup register budgets add up to the launch allocation:
+// 128 + 168 + 168 + 48 = 4 x 128 per thread (the build checks that ptxas
+// allocates 128 registers at entry).
+struct SfwCfg {
+  static constexpr int BN = 256;
+  static constexpr int NRB = 2;
+  static constexpr int A_BYTES = kBM * 128;
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int SFA_BYTES = 4 * 512;
+  static constexpr int SFB_BYTES = NRB * 4 * 512;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGES = (220 * 1024) / STAGE_BYTES;
+  static constexpr int NSF = 4;                       // TMEM scale buffers
+  static constexpr int SF_COLS = 16 + 16 * NRB;        // per buffer: 16 (A) + 32 (B)
+  static constexpr int SF_COL0 = BN;                   // after the accumulator
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+  static constexpr int THREADS = 512;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr uint32_t IDESC =
+      (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
+  static_assert(SF_COL0 + NSF * SF_COLS <= kTmemCols, "TMEM budget");
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+};
+
+__global__ void __launch_bounds__(SfwCfg::THREADS, 1)
+gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const GemmArgs args) {
+  using C = SfwCfg;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[C::STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
+  __shared__ __align__(8) uint64_t sff_bar[C::NSF];
+  __shared__ __align__(8) uint64_t sfe_bar[C::NSF];
+  __shared__ __align__(8) uint64_t accf_bar;
+  __shared__ __align__(8) uint64_t acce_bar;
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t s_tmem_base;
+  __shared__ volatile int s_abort;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int wg = warp >> 2;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < C::NSF; ++i) {
+      mbar_init(&sff_bar[i], 4);
+      mbar_init(&sfe_bar[i], 1);
+    }
+    mbar_init(&accf_bar, 1);
+    mbar_init(&acce_bar, C::EPI_WARPS);
+    mbar_init(&drain_bar, 1);
+    s_abort = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&s_tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
+        const Unit w = decode_unit(args, u);
+        for (int kt = w.kt0; kt < w.kt1; ++kt) {
+          if (!wait_or_abort(&empty_bar[stage], phase ^ 1u, args.budget, &s_abort)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          uint8_t* sb = sa + C::A_BYTES;
+          uint8_t* ssfa = sb + C::B_BYTES;
+          uint8_t* ssfb = ssfa + C::SFA_BYTES;
+          const int steps = min(4, args.k_steps - 4 * kt);
+          const int nrb = min(C::NRB, args.w_row_blocks - w.n * C::NRB);
+          mbar_arrive_expect_tx(&full_bar[stage],
+                                C::A_BYTES + C::B_BYTES + static_cast<uint32_t>(steps * 512 * (1 + nrb)));
+          armed |= 1u << stage;
+          armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+          tma_load_2d(sa, &tmA, &full_bar[stage], kt * 128, w.m * kBM);
+          tma_load_2d(sb, &tmB, &full_bar[stage], kt * 128, w.n * C::BN);
+          bulk_load(ssfa, args.xs + (static_cast<size_t>(w.m) * args.ka + 4 * kt) * 512, steps * 512,
+                    &full_bar[stage]);
+          for (int rb = 0; rb < nrb; ++rb)
+            bulk_load(ssfb + rb * 2048, args.ws + (static_cast<size_t>(w.n * C::NRB + rb) * args.ka + 4 * kt) * 512,
+                      steps * 512, &full_bar[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        for (int i = 0; i < C::STAGES; ++i)
+          if (armed & (1u << i)) {
+            const long long t0 = clock64();
+            while (!mbar_try_wait(&full_bar[i], (armed_phase >> i) & 1u) && clock64() - t0 < args.budget) {
+            }
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int sfb = 0;
+      uint32_t sf_phase = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
+        const Unit w = decode_unit(args, u);
+        if (!wait_or_abort(&acce_bar, acc_phase ^ 1u, args.budget, &s_abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kt = w.kt0; kt < w.kt1; ++kt) {
+          if (!wait_or_abort(&full_bar[stage], phase, args.budget, &s_abort) ||
+              !wait_or_abort(&sff_bar[sfb], sf_phase, args.budget, &s_abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sa + C::A_BYTES);
+          const uint32_t sf = tmem + C::SF_COL0 + sfb * C::SF_COLS;
+          const int steps = min(4, args.k_steps - 4 * kt);
+          for (int j = 0; j < steps; ++j)
+            mma_mxf4nvf4(tmem, sdesc_kmajor_sw128(a0 + 32 * j), sdesc_kmajor_sw128(b0 + 32 * j), C::IDESC,
+                         sf + 4 * j, sf + 16 + 8 * j, (kt > w.kt0 || j > 0) ? 1u : 0u);
+          umma_commit(&empty_bar[stage]);
+          umma_commit(&sfe_bar[sfb]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          if (++sfb == C::NSF) {
+            sfb = 0;
+            sf_phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&accf_bar);
+        acc_phase ^= 1u;
+      }
+      umma_commit(&drain_bar);
+      const long long t0 = clock64();
+      while (!mbar_try_wait(&drain_bar, 0) && clock64() - t0 < 4 * args.budget + 1000000) {
+      }
+    }
+  } else if (wg == 3) {
+    // ------------------------------------------------------ scale writers
+    regs_dec<48>();
+    const int q = warp & 3;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+    int stage = 0;
+    uint32_t phase = 0;
+    int sfb = 0;
+    uint32_t sf_phase = 0;
+    for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
+      const Unit w = decode_unit(args, u);
+      bool ok = true;
+      for (int kt = w.kt0; kt < w.kt1; ++kt) {
+        if (!wait_or_abort(&full_bar[stage], phase, args.budget, &s_abort) ||
+            !wait_or_abort(&sfe_bar[sfb], sf_phase ^ 1u, args.budget, &s_abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ssfa = smem_u32(smem + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES);
+        const uint32_t ssfb = ssfa + C::SFA_BYTES;
+        const uint32_t dst = tmem + lane_base + C::SF_COL0 + sfb * C::SF_COLS;
+        const int steps = min(4, args.k_steps - 4 * kt);
+        for (int j = 0; j < steps; ++j) {
+          tmem_st_32x32b_x4(dst + 4 * j, ld_shared_v4(ssfa + 512 * j + 16 * lane));
+#pragma unroll
+          for (int rb = 0; rb < C::NRB; ++rb)
+            tmem_st_32x32b_x4(dst + 16 + 8 * j + 4 * rb, ld_shared_v4(ssfb + rb * 2048 + 512 * j + 16 * lane));
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sff_bar[sfb]);
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        if (++sfb == C::NSF) {
+          sfb = 0;
+          sf_phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+    }
+    tmem_st_wait();
+  } else if (wg == 1 || wg == 2) {
+    // ------------------------------------------------------------ epilogue
+    regs_inc<168>();
+    const int e = warp - 4;
+    const int q = warp & 3;
+    const int h = e >> 2;
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
+      const Unit w = decode_unit(args, u);
+      if (!wait_or_abort(&accf_bar, acc_phase, args.budget, &s_abort)) break;
+      tc_fence_after();
+      const int row = w.m * kBM + 32 * q + lane;
+      const bool row_ok = row < args.M;
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(128 * h);
+      __syncwarp();
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tbase + 32 * c, r[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce_bar);
+      acc_phase ^= 1u;
+      const float rs = row_ok ? args.xg[row] * args.wg[0] : 0.0f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int col0 = w.n * C::BN + 128 * h + 32 * c;
+        if (row_ok && col0 < args.N) store_output<true>(args, row, col0, rs, r[c]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // Split-K reduction + epilogue: fixed split order, same scaling as the
 // direct epilogue.  8 outputs per thread.
 template <bool FP4>
@@ -513,11 +781,18 @@ cudaError_t run(const uint8_t* xq, const uint8_t* xs, const float* xg, const uin
   a.ka = static_cast<int>((K + 63) / 64);
   a.w_row_blocks = static_cast<int>((N + 127) / 128);
   a.budget = budget;
-  auto kern = gemm_kernel<FP4, BN>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-  if (e != cudaSuccess) return e;
   const int grid = plan.grid < a.units ? plan.grid : a.units;
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, a);
+  cudaError_t e;
+  if (FP4 && BN == 256) {
+    e = cudaFuncSetAttribute(gemm_fp4_sfw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SfwCfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    gemm_fp4_sfw_kernel<<<grid, SfwCfg::THREADS, SfwCfg::SMEM_BYTES, s>>>(ta, tb, a);
+  } else {
+    auto kern = gemm_kernel<FP4, BN>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, a);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess || plan.splits == 1) return e;
   const int64_t total8 = M * N / 8;
