@@ -129,11 +129,16 @@ __device__ __forceinline__ void store_partial(const GemmArgs& a, int split, int 
                                               const uint32_t (&r)[32]) {
   float* dst = a.partial + (static_cast<size_t>(split) * a.M + row) * a.N + col0;
   if (col0 + 32 <= a.N) {
+    if ((reinterpret_cast<uintptr_t>(dst) & 31u) == 0) {  // 32-byte stores need 32-byte alignment
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      reinterpret_cast<float4*>(dst)[j] =
-          make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                      __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+      for (int j = 0; j < 4; ++j) st_global_v8(dst + 8 * j, r + 8 * j);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        reinterpret_cast<float4*>(dst)[j] =
+            make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                        __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+    }
   } else {
 #pragma unroll
     for (int j = 0; j < 32; ++j)
@@ -173,11 +178,19 @@ __device__ __forceinline__ void store_output(const GemmArgs& a, int row, int col
     }
   }
   if (full) {
-    uint4* yp = reinterpret_cast<uint4*>(a.Y + base);
+    // two 32-byte stores: each thread writes whole sectors of its row
+    uint32_t pk[16];
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      yp[j] = make_uint4(pack_bf16x2(y[8 * j], y[8 * j + 1]), pack_bf16x2(y[8 * j + 2], y[8 * j + 3]),
-                         pack_bf16x2(y[8 * j + 4], y[8 * j + 5]), pack_bf16x2(y[8 * j + 6], y[8 * j + 7]));
+    for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(y[2 * j], y[2 * j + 1]);
+    __nv_bfloat16* yp = a.Y + base;
+    if ((reinterpret_cast<uintptr_t>(yp) & 31u) == 0) {  // 32-byte stores need 32-byte alignment
+      st_global_v8(yp, pk);
+      st_global_v8(yp + 16, pk + 8);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        reinterpret_cast<uint4*>(yp)[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+    }
   } else {
 #pragma unroll
     for (int j = 0; j < 32; ++j)
@@ -228,6 +241,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem_base;
+  // barrier setup, TMEM allocation and descriptor prefetch above overlap the
+  // previous kernel's tail; global memory is touched only after this wait
+  griddep_launch_dependents();
+  griddep_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -496,6 +513,10 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem_base;
+  // barrier setup, TMEM allocation and descriptor prefetch above overlap the
+  // previous kernel's tail; global memory is touched only after this wait
+  griddep_launch_dependents();
+  griddep_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -686,6 +707,8 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int spli
                                      const float* __restrict__ xg, const float* __restrict__ wg,
                                      const __nv_bfloat16* __restrict__ residual,
                                      __nv_bfloat16* __restrict__ Y) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int64_t idx8 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t total8 = static_cast<int64_t>(M) * N / 8;
   if (idx8 >= total8) return;
@@ -786,22 +809,20 @@ cudaError_t run(const uint8_t* xq, const uint8_t* xs, const float* xg, const uin
   if (FP4 && BN == 256) {
     e = cudaFuncSetAttribute(gemm_fp4_sfw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SfwCfg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    gemm_fp4_sfw_kernel<<<grid, SfwCfg::THREADS, SfwCfg::SMEM_BYTES, s>>>(ta, tb, a);
+    e = launch_pdl(gemm_fp4_sfw_kernel, dim3(grid), dim3(SfwCfg::THREADS), SfwCfg::SMEM_BYTES, s, ta, tb, a);
   } else {
     auto kern = gemm_kernel<FP4, BN>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, a);
+    e = launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, s, ta, tb, a);
   }
-  e = cudaGetLastError();
   if (e != cudaSuccess || plan.splits == 1) return e;
   const int64_t total8 = M * N / 8;
   const int threads = 256;
   const int64_t blocks = (total8 + threads - 1) / threads;
-  splitk_reduce_kernel<FP4><<<static_cast<unsigned int>(blocks), threads, 0, s>>>(
-      static_cast<const float*>(workspace), plan.splits, a.M, a.N, xg, wg,
-      static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(Y));
-  return cudaGetLastError();
+  return launch_pdl(splitk_reduce_kernel<FP4>, dim3(static_cast<unsigned int>(blocks)), dim3(threads), 0, s,
+                    static_cast<const float*>(workspace), plan.splits, a.M, a.N, xg, wg,
+                    static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(Y));
 }
 
 }  // namespace

@@ -216,6 +216,8 @@ template <int FMT, int MODE, int EPT>
 __global__ void __launch_bounds__(512, 1) quant_rows_plain_kernel(const RowArgs a) {
   constexpr int NB = EPT / 16;  // NVFP4 blocks per thread
   __shared__ float s_red[32];
+  griddep_launch_dependents();
+  griddep_wait();
   const int64_t row = blockIdx.x;
   const int t = threadIdx.x;
   const int K = a.K;
@@ -298,6 +300,8 @@ __global__ void __launch_bounds__(512, 1) quant_rows_xform_kernel(const RowArgs 
   extern __shared__ uint4 s_row[];
   __shared__ float s_red[32];
   __shared__ float s_r;
+  griddep_launch_dependents();
+  griddep_wait();
 
   const int64_t row = blockIdx.x;
   const int b = threadIdx.x;
@@ -412,6 +416,8 @@ __global__ void __launch_bounds__(512, 1) quant_rows_xform_kernel(const RowArgs 
 }
 
 __global__ void finalize_global_kernel(float* g) {
+  griddep_launch_dependents();
+  griddep_wait();
   g[0] = __fdiv_rn(__uint_as_float(*reinterpret_cast<unsigned int*>(g)), 2688.0f);
 }
 
@@ -443,11 +449,9 @@ cudaError_t launch_rows(const void* X, int64_t rows, int64_t K, const void* gamm
     // one NVFP4 block per thread while a row fits in 512 threads
     if (K <= 8192) {
       const int threads = static_cast<int>(((K + 63) / 64 * 4 + 31) / 32 * 32);
-      quant_rows_plain_kernel<FMT, MODE, 16><<<grid, threads, 0, s>>>(a);
-    } else {
-      quant_rows_plain_kernel<FMT, MODE, 64><<<grid, threads_for(K), 0, s>>>(a);
+      return launch_pdl(quant_rows_plain_kernel<FMT, MODE, 16>, dim3(grid), dim3(threads), 0, s, a);
     }
-    return cudaGetLastError();
+    return launch_pdl(quant_rows_plain_kernel<FMT, MODE, 64>, dim3(grid), dim3(threads_for(K)), 0, s, a);
   }
   // staged bf16 row, rounded up to whole 64-element groups (the chunk
   // swizzle permutes within groups of 8 chunks)
@@ -457,8 +461,7 @@ cudaError_t launch_rows(const void* X, int64_t rows, int64_t K, const void* gamm
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  kern<<<grid, threads_for(K), smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(threads_for(K)), smem, s, a);
 }
 
 }  // namespace
@@ -482,8 +485,7 @@ cudaError_t launch_quant_weight_nvfp4(const void* W, int64_t N, int64_t K, uint3
   e = launch_rows<kNvfp4, kTensorQuant>(W, N, K, nullptr, 0.0f, f, codes, nvfp4_code_pitch(K), scales, nullptr,
                                         amax, s);
   if (e != cudaSuccess) return e;
-  finalize_global_kernel<<<1, 1, 0, s>>>(g_w);
-  return cudaGetLastError();
+  return launch_pdl(finalize_global_kernel, dim3(1), dim3(1), 0, s, g_w);
 }
 
 cudaError_t launch_quant_fp8(const void* X, int64_t rows, int64_t K, const void* gamma, float eps, uint32_t flags,
