@@ -52,7 +52,7 @@ def test_noalloc_matches_workspace_path_twice(M, N, K, residual):
 def test_noalloc_direct_path_without_split():
     """A prefill-sized shape needs no scratch and must still work."""
     m = vq()
-    M, N, K = 1024, 1280, 512
+    M, N, K = 1024, 2560, 512
     assert m.vlaq_linear_workspace_bytes(M, N, K) == 0
     xq, xs, xg, wq, ws, wg, _ = _case(m, M, N, K, 303, False)
     Y_ref = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")

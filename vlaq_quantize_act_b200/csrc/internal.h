@@ -40,6 +40,10 @@ struct GemmPlan {
   size_t ws_bytes; // fp32 partials needed when splits > 1
 };
 GemmPlan plan_gemm(bool fp4, int64_t M, int64_t N, int64_t K, int num_sms);
+// fp32 partial sums of a split-K plan, rounded up to 256 bytes.
+inline size_t splitk_partial_bytes(int64_t splits, int64_t M, int64_t N) {
+  return (static_cast<size_t>(splits) * M * N * sizeof(float) + 255) / 256 * 256;
+}
 
 cudaError_t launch_linear(bool fp4, const uint8_t* xq, const uint8_t* xs, const float* xg,
                           const uint8_t* wq, const uint8_t* ws, const float* wg,
