@@ -96,7 +96,6 @@ vlaq_status check_flags(const char* fn, uint32_t flags, uint32_t allowed) {
   return VLAQ_OK;
 }
 
-constexpr long long kDefaultBudget = 2000000000LL;  // ~1 s of SM clock per wait
 
 }  // namespace
 
@@ -117,6 +116,10 @@ vlaq_status vlaq_check(void* stream) {
   unsigned int st = 0;
   cudaError_t e = vlaq::read_and_clear_status(&st, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail("vlaq_check", e);
+  unsigned int qst = 0;
+  e = vlaq::read_and_clear_quant_status(&qst, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail("vlaq_check", e);
+  st |= qst;
   if (st & vlaq::kStatusTimeout)
     return fail(VLAQ_ERR_TIMEOUT, "vlaq_check: a kernel gave up a bounded wait (device status 0x%x)", st);
   return ok();
@@ -236,7 +239,7 @@ static vlaq_status linear_common(const char* fn, bool fp4, const uint8_t* xq, co
     if (!aligned16(workspace)) return fail(VLAQ_ERR_ALIGN, "%s: workspace is not 16-byte aligned", fn);
   }
   cudaError_t e = vlaq::launch_linear(fp4, xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, ws_bytes, plan,
-                                      kDefaultBudget, static_cast<cudaStream_t>(stream));
+                                      vlaq::kWaitBudgetCycles, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(fn, e);
   return ok();
 }

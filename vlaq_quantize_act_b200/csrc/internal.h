@@ -13,8 +13,11 @@ namespace vlaq {
 // Device status word bits (read and cleared by vlaq_check).
 enum : unsigned int { kStatusTimeout = 1u };
 
-// Largest K the one-thread-per-64-block prologue supports (512 threads).
+// Largest K of the row quantizers: two staged bf16 rows (2 x 64 KiB) per CTA.
 constexpr int64_t kMaxQuantK = 32768;
+
+// Clock-cycle limit of every bounded wait in the library kernels (~1 s).
+constexpr long long kWaitBudgetCycles = 2000000000LL;
 
 constexpr uint32_t kFlagRmsNorm = 1u;
 constexpr uint32_t kFlagHadamard = 2u;
@@ -51,8 +54,9 @@ cudaError_t launch_linear(bool fp4, const uint8_t* xq, const uint8_t* xs, const 
                           void* workspace, size_t ws_bytes, const GemmPlan& plan,
                           long long wait_budget, cudaStream_t s);
 
-// Device status word accessors (gemm.cu).
+// Device status word accessors (gemm.cu, quant.cu).
 cudaError_t read_and_clear_status(unsigned int* out, cudaStream_t s);
+cudaError_t read_and_clear_quant_status(unsigned int* out, cudaStream_t s);
 
 // Kernel launch with the programmatic-stream-serialization attribute, so the
 // kernel may start while the previous kernel on the stream drains; every

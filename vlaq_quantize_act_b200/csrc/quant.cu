@@ -1,44 +1,59 @@
 // Fused activation prologue and the offline weight quantizers.
 //
-// One CTA per row; thread b owns the 64-element block b of the row (the
-// Hadamard block, four NVFP4 scale blocks, 32 packed code bytes and one
-// 4-byte word of the 128x4 tiled scale layout).  The row is read once from
-// HBM with 16-byte loads, optionally transformed in registers (RMSNorm,
-// block-64 WHT), reduced to a per-row amax with warp shuffles, then
-// quantized and written with 16-byte stores.  HBM-bound: 2 bytes in and
-// 0.5625 (NVFP4) or 1 (FP8) bytes out per element.
+// Persistent CTAs, several per SM, each keeping up to four rows in flight in
+// a shared-memory ring: thread 0 fetches a whole bf16 row with one bulk copy
+// (cp.async.bulk, completion on the slot's mbarrier) and the CTA quantizes
+// the oldest staged row while the next ones stream in, so HBM sees a steady
+// queue of large reads instead of one dependent load-reduce-store chain per
+// row.  A staged row is read twice from shared memory:
+//   pass A  (transform and) per-16 block amax, kept in registers; row amax
+//           -> global scale g of the row;
+//   pass B  transform again, E4M3 block scale, codes.
+// Lane l of warp w owns the 16-element block 32 (W it + w) + l of the row (W
+// warps per CTA): one NVFP4 scale byte and 8 code bytes, so four lanes hold
+// one Hadamard block and one 4-byte word of the 128x4 tiled scale layout,
+// and a warp writes 256 (NVFP4) or 512 (FP8) contiguous code bytes per step.
+// HBM-bound: 2 bytes in and 0.5625 (NVFP4) or 1 (FP8) bytes out per element.
+// Short rows (K <= 8192) run 8-warp CTAs, four per SM; long rows 16-warp
+// CTAs, two per SM, so one row is spread over more lanes.
 //
 // Arithmetic follows the format definitions stated in include/vlaq.h: every
 // fp32 operation is an explicitly rounded intrinsic (no contraction),
 // division and square root are correctly rounded, so codes and scales are
 // bit-identical to any implementation that performs the same operations
 // ("FoldQuant W8A8/W4A4 inference", SYCL commit: correctly rounded divide
-// and sqrt, fixed reduction tree).
+// and sqrt, fixed reduction tree).  The RMSNorm sum of squares follows the
+// fixed 32-lane tree (lane l accumulates the 8-element chunks l, l + 32, ...
+// in order with fused multiply-adds, then an XOR butterfly), and the
+// Hadamard butterfly keeps the sequential stage order h = 1, 2, ..., 32.
 //
-// Fast exact quotient: the code of x / S only depends on which side of the
-// format's rounding decision points the correctly rounded quotient falls.
-// Every decision point of E2M1 (the grid midpoints 0.25 ... 5) has its low
-// 21 fp32 mantissa bits zero, and every decision point of E4M3 its low 19.
-// q' = x * RN(1/S) is within 3 units in the last place of x / S, so when q'
-// is more than 8 units away from any number with those low bits zero, q'
-// and RN(x / S) give the same code; otherwise (a few per million elements,
-// and values that sit exactly on grid-like numbers) the 16 values of the
-// block are divided exactly.
+// Every quotient x / S is the correctly rounded one (Markstein's
+// correction step after a product with the correctly rounded reciprocal,
+// see quotients() below), so the codes equal those of a plain division.
 #include <cuda_bf16.h>
 
 #include "internal.h"
 #include "ptx.cuh"
 
 namespace vlaq {
+
+__device__ unsigned int g_vlaq_quant_status = 0;
+
 namespace {
 
 enum { kNvfp4 = 0, kFp8 = 1 };
 enum { kPerRow = 0, kTensorAmax = 1, kTensorQuant = 2 };
 
-// XOR swizzle of 16-byte chunks in the staged row: both the per-thread
-// writes (8 consecutive chunks) and the lane-strided tree reads hit 8
-// distinct 16-byte bank groups.
-__device__ __forceinline__ int swz_chunk(int c) { return c ^ ((c >> 3) & 7); }
+constexpr int kMaxRowBufs = 4;
+constexpr int kShortRowK = 8192;  // rows up to this length take the 8-warp CTAs
+
+// CTA shape per row length: W warps, CTAs resident per SM, ring budget.
+template <int W>
+struct RowCfg {
+  static constexpr int kThreads = 32 * W;
+  static constexpr int kCtasPerSm = 1024 / kThreads;  // 32 warps per SM, 64 registers a thread
+  static constexpr int kRingBytes = (W == 8) ? 52 * 1024 : 110 * 1024;
+};
 
 __device__ __forceinline__ void unpack_bf16x8(const uint4& q, float* v) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
@@ -49,26 +64,101 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& q, float* v) {
   }
 }
 
-// max |x| of 16 bf16 values held in two 16-byte words (exact).
+// max |x| of 16 bf16 values (two 16-byte words), exact: kept packed as
+// bf16 pairs, the max of bf16 values is one of them.
 __device__ __forceinline__ float absmax_bf16x16(const uint4& a, const uint4& b) {
   const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-  const uint32_t zero = 0u;
-  __nv_bfloat162 m = *reinterpret_cast<const __nv_bfloat162*>(&zero);
+  __nv_bfloat162 h[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const uint32_t aw = w[j] & 0x7FFF7FFFu;  // |x| of both halves
-    m = __hmax2(m, *reinterpret_cast<const __nv_bfloat162*>(&aw));
+    h[j] = *reinterpret_cast<const __nv_bfloat162*>(&aw);
   }
-  return fmaxf(__low2float(m), __high2float(m));
+#pragma unroll
+  for (int s = 4; s; s >>= 1)
+#pragma unroll
+    for (int j = 0; j < s; ++j) h[j] = __hmax2(h[j], h[j + s]);
+  return fmaxf(__low2float(h[0]), __high2float(h[0]));
 }
 
-// Normalised Walsh-Hadamard transform of one 64-block, Sylvester order:
-// butterfly stages h = 1, 2, ..., 32, then x 1/8 (exact).
-__device__ __forceinline__ void wht64(float* v) {
+// Correctly rounded quotient without a divide per element: Markstein's
+// correction step (P. Markstein, "IA-64 and Elementary Functions", 2000:
+// with y = RN(1/S) and q0 = RN(x y), the residual x - q0 S is exact under a
+// fused multiply-add and RN(q0 + (x - q0 S) y) = RN(x / S)).  The residual
+// is formed negated, e' = q0 S - x, so that x = -0 still yields -0.  The
+// reciprocal is CUDA's correctly rounded __frcp_rn, once per divisor.  Only
+// divisors far from 1 (where the residual or 1/S could leave the normal
+// range) and S = 0 take the slow path, behind a warp vote.
+struct Divisor {
+  float S, y;
+  bool slow;  // S = 0 (quotients 0) or S outside [2^-64, 2^64]
+};
+
+__device__ __forceinline__ Divisor make_divisor(float S) {
+  Divisor d;
+  d.S = S;
+  const bool ok = S >= 0x1p-64f && S <= 0x1p64f;
+  d.y = ok ? __frcp_rn(S) : 0.0f;
+  d.slow = !ok;
+  return d;
+}
+
+__device__ __forceinline__ float markstein_quotient(float x, float S, float y) {
+  const float q0 = __fmul_rn(x, y);
+  const float e = __fmaf_rn(q0, S, -x);  // q0 S - x, exact
+  return __fmaf_rn(-e, y, q0);
+}
+
+// RN(v[i] / S) for N values (0 when S = 0).  Executed by the whole warp.
+template <int N>
+__device__ __forceinline__ void quotients(const float* v, const Divisor& d, float* q) {
 #pragma unroll
-  for (int h = 1; h < 64; h <<= 1) {
+  for (int i = 0; i < N; ++i) q[i] = markstein_quotient(v[i], d.S, d.y);
+  if (__any_sync(0xffffffffu, d.slow)) {
+    if (d.slow) {
 #pragma unroll
-    for (int i = 0; i < 64; ++i) {
+      for (int i = 0; i < N; ++i) q[i] = (d.S == 0.0f) ? 0.0f : __fdiv_rn(v[i], d.S);
+    }
+  }
+}
+
+// E4M3 byte of RN(a / d) for a >= 0 (d is warp-uniform).
+__device__ __forceinline__ uint32_t e4m3_of_quotient(float a, const Divisor& d) {
+  const float q = d.slow ? __fdiv_rn(a, d.S) : markstein_quotient(a, d.S, d.y);
+  return cvt_e4m3x2(q, 0.0f) & 0xFFu;
+}
+
+// Byte offset of (row, 64-block 0) in the 128x4 tiled scale layout
+// (512-byte atom per 128 rows x 4 blocks; nblk = 64-blocks per row).
+__device__ __forceinline__ int64_t scale_row_base(int64_t row, int nblk) {
+  return (row >> 7) * nblk * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4;
+}
+
+struct RowArgs {
+  const __nv_bfloat16* X;
+  int K;
+  const __nv_bfloat16* gamma;
+  float eps;
+  uint8_t* codes;
+  int64_t pitch;
+  uint8_t* scales;
+  float* gout;
+  unsigned int* amax_word;
+  int64_t rows;
+  int nbuf;       // ring depth (rows in flight per CTA)
+  int row_bytes;  // ring slot size (2 K rounded up to 128)
+  long long budget;
+};
+
+// Normalised WHT of the 64-block spread over lanes 4 g .. 4 g + 3 (16 values
+// each, element 16 (lane % 4) + j): stages h = 1, 2, 4, 8 inside the lane,
+// h = 16, 32 across lanes (xor 1, 2), then x 1/8 (exact) -- the stages of the
+// sequential butterfly in the same order.  Executed by the whole warp.
+__device__ __forceinline__ void wht64_lanes(float* v, int lane) {
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
       if ((i & h) == 0) {
         const float a = v[i], b = v[i + h];
         v[i] = __fadd_rn(a, b);
@@ -77,340 +167,231 @@ __device__ __forceinline__ void wht64(float* v) {
     }
   }
 #pragma unroll
-  for (int i = 0; i < 64; ++i) v[i] = __fmul_rn(v[i], 0.125f);
-}
-
-// Max over the CTA; every thread gets the result.
-__device__ __forceinline__ float block_max(float v, float* s_red) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  if (l == 0) s_red[w] = v;
-  __syncthreads();
-  const int nw = blockDim.x >> 5;
-  float r = (l < nw) ? s_red[l] : 0.0f;
-#pragma unroll
-  for (int o = 16; o; o >>= 1) r = fmaxf(r, __shfl_xor_sync(0xffffffffu, r, o));
-  return r;
-}
-
-// Fast path of the quotient (see the file comment): approximate reciprocal
-// (at most 2 units in the last place off, documented bound of
-// rcp.approx.f32), one product per element, and a test that the product is
-// at least 8 units in the last place away from every number whose low
-// LOWBITS mantissa bits are zero.  t = (bits + 8) & (low mask without the
-// last 4 bits) is zero exactly for products within [-8, +7] units of such a
-// number (+-0 included, which merely takes the exact path).
-__device__ __forceinline__ float rcp_approx(float x) {
-  float r;
-  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
-}
-
-template <int LOWBITS>
-__device__ __forceinline__ uint32_t near_key(float q) {
-  return (__float_as_uint(q) + 8u) & (((1u << LOWBITS) - 1u) & ~0xFu);
-}
-
-// The reciprocal shortcut needs 1/S to be a normal fp32 number.
-__device__ __forceinline__ bool rcp_ok(float s) { return s >= 0x1p-125f && s <= 0x1p125f; }
-
-// RN(v[i] / S) for 16 values, S > 0, as far as E2M1 (LOWBITS = 21) or E4M3
-// (LOWBITS = 19) encoding can tell.  r = approximate 1/S, fast = rcp_ok(S).
-template <int LOWBITS>
-__device__ __forceinline__ void quotients16(const float* v, float S, float r, bool fast, float* q) {
-  uint32_t key = fast ? 0xFFFFFFFFu : 0u;
-  if (fast) {
+  for (int x = 1; x < 4; x <<= 1) {
+    const bool upper = (lane & x) != 0;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      q[i] = __fmul_rn(v[i], r);
-      key = min(key, near_key<LOWBITS>(q[i]));
+      const float p = __shfl_xor_sync(0xffffffffu, v[i], x);
+      v[i] = upper ? __fsub_rn(p, v[i]) : __fadd_rn(v[i], p);
     }
   }
-  if (key == 0u) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(v[i], S);
-  }
+  for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], 0.125f);
 }
 
-// E4M3 byte of RN(a / d) (a >= 0, d > 0) with r_d = approximate 1/d.
-__device__ __forceinline__ uint32_t e4m3_of_quotient(float a, float d, float r_d, bool fast) {
-  float q = fast ? __fmul_rn(a, r_d) : 0.0f;
-  if (!fast || near_key<19>(q) == 0u) q = __fdiv_rn(a, d);
-  return cvt_e4m3x2(q, 0.0f) & 0xFFu;
-}
-
-// Scale byte and 16 codes (two words) of one NVFP4 block.
-__device__ __forceinline__ uint32_t nvfp4_block(const float* v, float a16, float g, float six_g, float r6g,
-                                                bool fast6g, uint32_t& w0, uint32_t& w1) {
-  float q[16];
-  uint32_t sb8 = 0;
-  float S = 0.0f;
-  if (g > 0.0f) {
-    sb8 = e4m3_of_quotient(a16, six_g, r6g, fast6g);
-    S = __fmul_rn(e4m3_to_f32(sb8), g);
-  }
-  if (S != 0.0f) {
-    const bool fast = rcp_ok(S);
-    quotients16<21>(v, S, fast ? rcp_approx(S) : 0.0f, fast, q);
-  } else {
+// The 16 values of block q after the row transform (zeros past the row):
+// y = (x r) gamma for RMSNorm, then the block-64 WHT.  Warp-uniform.
+template <bool NORM, bool WHT>
+__device__ __forceinline__ void block_values(const RowArgs& a, const uint8_t* rs, int q, int nblk16, float r,
+                                             int lane, float* v) {
+  if (q < nblk16) {
+    const uint4* src = reinterpret_cast<const uint4*>(rs) + 2 * q;
+    unpack_bf16x8(src[0], v);
+    unpack_bf16x8(src[1], v + 8);
+    if (NORM) {
+      const uint4* gsrc = reinterpret_cast<const uint4*>(a.gamma) + 2 * q;
+      float gm[16];
+      unpack_bf16x8(__ldg(gsrc), gm);
+      unpack_bf16x8(__ldg(gsrc + 1), gm + 8);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) q[i] = 0.0f;
-  }
-  w0 = cvt_e2m1x8(q);
-  w1 = cvt_e2m1x8(q + 8);
-  return sb8;
-}
-
-// 16 FP8 codes (four words) with the row scale s.
-__device__ __forceinline__ void fp8_block(const float* v, float s, float r, bool fast, uint32_t* w) {
-  float q[16];
-  if (s != 0.0f) {
-    quotients16<19>(v, s, r, fast, q);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) q[i] = 0.0f;
-  }
-#pragma unroll
-  for (int j = 0; j < 4; ++j) w[j] = cvt_e4m3x2(q[4 * j], q[4 * j + 1]) | (cvt_e4m3x2(q[4 * j + 2], q[4 * j + 3]) << 16);
-}
-
-__device__ __forceinline__ void store_scale_word(uint8_t* scales, int64_t row, int b, int nblk, uint32_t word) {
-  // 128x4 tiled scale layout: 512-byte atom per (128 rows, 4 blocks)
-  const int64_t atom = (row >> 7) * nblk + b;
-  const int64_t off = atom * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4;
-  *reinterpret_cast<uint32_t*>(scales + off) = word;
-}
-
-struct RowArgs {
-  const __nv_bfloat16* X;
-  int K;
-  const __nv_bfloat16* gamma;
-  float eps;
-  uint32_t flags;
-  uint8_t* codes;
-  int64_t pitch;
-  uint8_t* scales;
-  float* gout;
-  unsigned int* amax_word;
-};
-
-// Global scale of the row (per-row modes) or of the tensor (quant pass).
-template <int FMT, int MODE>
-__device__ __forceinline__ float row_global(const RowArgs& a, float local, float* s_red, int64_t row) {
-  if (MODE == kPerRow) {
-    const float A = block_max(local, s_red);
-    const float g = (FMT == kNvfp4) ? __fdiv_rn(A, 2688.0f) : __fdiv_rn(A, 448.0f);
-    if (threadIdx.x == 0) a.gout[row] = g;
-    return g;
-  }
-  return __fdiv_rn(__uint_as_float(*a.amax_word), 2688.0f);
-}
-
-// ---- rows without RMSNorm / Hadamard.  Thread t owns the elements
-// [EPT t, EPT t + EPT) of the row (EPT = 16: one NVFP4 block, EPT = 64: one
-// 64-block); the raw bf16 stays packed in registers.  Small EPT gives short
-// rows many more warps in flight.  Threads past K / EPT (up to the next
-// multiple of 64 elements) write the zero padding of codes and scales.
-template <int FMT, int MODE, int EPT>
-__global__ void __launch_bounds__(512, 1) quant_rows_plain_kernel(const RowArgs a) {
-  constexpr int NB = EPT / 16;  // NVFP4 blocks per thread
-  __shared__ float s_red[32];
-  griddep_launch_dependents();
-  griddep_wait();
-  const int64_t row = blockIdx.x;
-  const int t = threadIdx.x;
-  const int K = a.K;
-  const int nblk64 = (K + 63) >> 6;
-  const int nel = max(0, min(EPT, K - EPT * t));         // real elements of this thread
-  const bool writes = EPT * t < 64 * nblk64;             // inside the padded row
-
-  const uint4* xr = reinterpret_cast<const uint4*>(a.X + row * static_cast<int64_t>(K));
-  uint4 raw[2 * NB];
-#pragma unroll
-  for (int i = 0; i < 2 * NB; ++i)
-    raw[i] = (8 * i < nel) ? __ldg(xr + (EPT / 8) * t + i) : make_uint4(0, 0, 0, 0);
-  float a16[NB];
-  float local = 0.0f;
-#pragma unroll
-  for (int q = 0; q < NB; ++q) {
-    a16[q] = absmax_bf16x16(raw[2 * q], raw[2 * q + 1]);
-    local = fmaxf(local, a16[q]);
-  }
-
-  if (MODE == kTensorAmax) {
-    const float A = block_max(local, s_red);
-    if (threadIdx.x == 0) atomicMax(a.amax_word, __float_as_uint(A));  // A >= 0: bit order = value order
-    return;
-  }
-  const float g = row_global<FMT, MODE>(a, local, s_red, row);
-
-  if (FMT == kNvfp4) {
-    const float six_g = __fmul_rn(6.0f, g);
-    const bool fast6g = rcp_ok(six_g);
-    const float r6g = fast6g ? rcp_approx(six_g) : 0.0f;
-    uint32_t sc_word = 0;
-    uint32_t cw[2 * NB];
-#pragma unroll
-    for (int q = 0; q < NB; ++q) {
-      cw[2 * q] = cw[2 * q + 1] = 0u;
-      if (16 * q < nel) {
-        float v[16];
-        unpack_bf16x8(raw[2 * q], v);
-        unpack_bf16x8(raw[2 * q + 1], v + 8);
-        const uint32_t sb8 = nvfp4_block(v, a16[q], g, six_g, r6g, fast6g, cw[2 * q], cw[2 * q + 1]);
-        sc_word |= sb8 << (8 * ((EPT == 16 ? t : q) & 3));
-      }
-    }
-    if (EPT == 16) {
-      // four neighbouring threads own the four bytes of one scale word
-      sc_word |= __shfl_xor_sync(0xffffffffu, sc_word, 1);
-      sc_word |= __shfl_xor_sync(0xffffffffu, sc_word, 2);
-      if (writes) {
-        *reinterpret_cast<uint2*>(a.codes + row * a.pitch + 8 * t) = make_uint2(cw[0], cw[1]);
-        if ((t & 3) == 0) store_scale_word(a.scales, row, t >> 2, nblk64, sc_word);
-      }
-    } else if (writes) {
-      uint4* crow = reinterpret_cast<uint4*>(a.codes + row * a.pitch + 32 * t);
-      crow[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-      crow[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-      store_scale_word(a.scales, row, t, nblk64, sc_word);
+      for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(__fmul_rn(v[j], r), gm[j]);
     }
   } else {
-    const bool fast = rcp_ok(g);
-    const float r = fast ? rcp_approx(g) : 0.0f;
-    uint4* crow = reinterpret_cast<uint4*>(a.codes + row * a.pitch + EPT * t);
 #pragma unroll
-    for (int q = 0; q < NB; ++q) {
-      if (16 * q < nel) {
-        float v[16];
-        unpack_bf16x8(raw[2 * q], v);
-        unpack_bf16x8(raw[2 * q + 1], v + 8);
-        uint32_t w[4];
-        fp8_block(v, g, r, fast, w);
-        crow[q] = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    }
+    for (int j = 0; j < 16; ++j) v[j] = 0.0f;
   }
+  if (WHT) wht64_lanes(v, lane);
 }
 
-// ---- rows with RMSNorm and / or the block-64 Hadamard rotation
-template <int FMT, int MODE>
-__global__ void __launch_bounds__(512, 1) quant_rows_xform_kernel(const RowArgs a) {
-  extern __shared__ uint4 s_row[];
-  __shared__ float s_red[32];
+__device__ __forceinline__ float absmax16(const float* v) {
+  float m = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) m = fmaxf(m, fabsf(v[j]));
+  return m;
+}
+
+// All rows of one launch: FMT (NVFP4 / FP8), MODE (per-row scale, tensor
+// amax pass, tensor quantize pass), NORM (RMSNorm, per-row modes only), WHT
+// (block-64 Hadamard), W warps per CTA.  Persistent grid: the CTA takes rows
+// blockIdx.x + i gridDim.x, the ring slot of row i is i mod nbuf.
+template <int FMT, int MODE, bool NORM, bool WHT, int W>
+__global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) quant_rows_kernel(const RowArgs a) {
+  constexpr int T = RowCfg<W>::kThreads;
+  constexpr int MAXIT = (W == 8 ? kShortRowK : int(kMaxQuantK)) / 16 / T;  // blocks per lane, at most
+  extern __shared__ __align__(128) uint8_t s_ring[];
+  __shared__ __align__(8) uint64_t s_bar[kMaxRowBufs];
+  __shared__ float s_red[W];
   __shared__ float s_r;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int K = a.K;
+  const int nblk16 = K >> 4;
+  const int nblk64 = (K + 63) >> 6;
+  const int nblk16_pad = 4 * nblk64;  // blocks up to the padded row end
+  const int iters = (nblk16_pad + T - 1) / T;
+  const int nbuf = a.nbuf;
+  const uint32_t row_tx = static_cast<uint32_t>(2 * K);
+  const int64_t stride = gridDim.x;
+
+  if (tid == 0) {
+    for (int b = 0; b < nbuf; ++b) mbar_init(&s_bar[b], 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
   griddep_launch_dependents();
   griddep_wait();
 
-  const int64_t row = blockIdx.x;
-  const int b = threadIdx.x;
-  const int K = a.K;
-  const int nblk = (K + 63) >> 6;
-  const bool active = b < nblk;
-  const int nel = active ? min(64, K - 64 * b) : 0;
-  const bool do_norm = (MODE == kPerRow) && (a.flags & kFlagRmsNorm);
-  const bool do_wht = (a.flags & kFlagHadamard) != 0;
-
-  // ---- load the 64-block (bf16 -> fp32 is exact)
-  const uint4* xr = reinterpret_cast<const uint4*>(a.X + row * static_cast<int64_t>(K));
-  float v[64];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    if (8 * i < nel) {
-      const uint4 q = __ldg(xr + 8 * b + i);
-      unpack_bf16x8(q, v + 8 * i);
-      if (do_norm) s_row[swz_chunk(8 * b + i)] = q;
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[8 * i + j] = 0.0f;
+  if (tid == 0) {
+    for (int b = 0; b < nbuf; ++b) {
+      const int64_t row = blockIdx.x + b * stride;
+      if (row >= a.rows) break;
+      mbar_arrive_expect_tx(&s_bar[b], row_tx);
+      bulk_load(s_ring + b * a.row_bytes, a.X + row * K, row_tx, &s_bar[b]);
     }
   }
+  float g_tensor = 0.0f;
+  if (MODE == kTensorQuant) g_tensor = __fdiv_rn(__uint_as_float(*a.amax_word), 2688.0f);
 
-  // ---- RMSNorm: fixed 32-lane tree over the staged row, then y = (x r) g
-  if (do_norm) {
+  int slot = 0;
+  uint32_t phase = 0;
+  for (int64_t row = blockIdx.x; row < a.rows; row += stride) {
+    const bool ok = __syncthreads_and(mbar_wait(&s_bar[slot], phase, a.budget));
+    if (!ok) {
+      // record it, let the copies still in flight land, and stop
+      if (tid == 0) {
+        atomicOr(&g_vlaq_quant_status, kStatusTimeout);
+        for (int k = 0; k < nbuf && row + k * stride < a.rows; ++k) {
+          const int sk = slot + k;
+          mbar_wait(&s_bar[sk % nbuf], phase ^ (sk >= nbuf ? 1u : 0u), a.budget);
+        }
+      }
+      break;
+    }
+    const uint8_t* rs = s_ring + slot * a.row_bytes;
+
+    // ---- RMSNorm factor r = 1 / sqrt(mean(x^2) + eps), fixed 32-lane tree
+    float r = 1.0f;
+    if (NORM) {
+      if (warp == 0) {
+        float acc = 0.0f;
+        for (int c = lane; c < (K >> 3); c += 32) {
+          float t[8];
+          unpack_bf16x8(reinterpret_cast<const uint4*>(rs)[c], t);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc = __fmaf_rn(t[j], t[j], acc);
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
+        if (lane == 0) {
+          const float mean = __fdiv_rn(acc, static_cast<float>(K));
+          s_r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean, a.eps)));
+        }
+      }
+      __syncthreads();
+      r = s_r;
+    }
+
+    // ---- pass A: per-block amax (kept in registers) and row amax
+    float a16r[MAXIT];
+    float g = g_tensor;
+    if (MODE != kTensorQuant) {
+      float local = 0.0f;
+#pragma unroll
+      for (int it = 0; it < MAXIT; ++it) {
+        a16r[it] = 0.0f;
+        if (it < iters) {
+          const int q = (it * W + warp) * 32 + lane;
+          float m = 0.0f;
+          if (NORM || WHT) {
+            float v[16];
+            block_values<NORM, WHT>(a, rs, q, nblk16, r, lane, v);
+            m = absmax16(v);
+          } else if (q < nblk16) {
+            const uint4* src = reinterpret_cast<const uint4*>(rs) + 2 * q;
+            m = absmax_bf16x16(src[0], src[1]);
+          }
+          a16r[it] = m;
+          local = fmaxf(local, m);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) local = fmaxf(local, __shfl_xor_sync(0xffffffffu, local, o));
+      if (lane == 0) s_red[warp] = local;
+      __syncthreads();
+      float A = s_red[0];
+#pragma unroll
+      for (int w = 1; w < W; ++w) A = fmaxf(A, s_red[w]);
+      if (MODE == kTensorAmax) {
+        if (tid == 0) atomicMax(a.amax_word, __float_as_uint(A));  // A >= 0: bit order = value order
+      } else {
+        g = (FMT == kNvfp4) ? __fdiv_rn(A, 2688.0f) : __fdiv_rn(A, 448.0f);
+        if (tid == 0) a.gout[row] = g;
+      }
+    }
+
+    // ---- pass B: block scales and codes
+    if (MODE != kTensorAmax) {
+      uint8_t* crow = a.codes + row * a.pitch;
+      if (FMT == kNvfp4) {
+        uint8_t* srow = a.scales + scale_row_base(row, nblk64);
+        const Divisor d6g = make_divisor(__fmul_rn(6.0f, g));
+#pragma unroll
+        for (int it = 0; it < MAXIT; ++it) {
+          if (it < iters) {
+            const int q = (it * W + warp) * 32 + lane;
+            float v[16];
+            block_values<NORM, WHT>(a, rs, q, nblk16, r, lane, v);
+            const float a16 = (MODE == kPerRow) ? a16r[it] : absmax16(v);
+            uint32_t sb8 = 0;
+            float S = 0.0f;
+            if (g > 0.0f) {
+              sb8 = e4m3_of_quotient(a16, d6g);
+              S = __fmul_rn(e4m3_to_f32(sb8), g);
+            }
+            const Divisor dv = make_divisor(S);
+            float qv[16];
+            quotients<16>(v, dv, qv);
+            const uint32_t w0 = cvt_e2m1x8(qv);
+            const uint32_t w1 = cvt_e2m1x8(qv + 8);
+            if (q < nblk16_pad) {
+              *reinterpret_cast<uint2*>(crow + 8 * q) = make_uint2(w0, w1);
+              srow[(q >> 2) * 512 + (q & 3)] = static_cast<uint8_t>(sb8);
+            }
+          }
+        }
+      } else {
+        const Divisor dg = make_divisor(g);
+#pragma unroll
+        for (int it = 0; it < MAXIT; ++it) {
+          if (it < iters) {
+            const int q = (it * W + warp) * 32 + lane;
+            float v[16];
+            block_values<NORM, WHT>(a, rs, q, nblk16, r, lane, v);
+            float qv[16];
+            quotients<16>(v, dg, qv);
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              w[j] = cvt_e4m3x2(qv[4 * j], qv[4 * j + 1]) | (cvt_e4m3x2(qv[4 * j + 2], qv[4 * j + 3]) << 16);
+            if (q < nblk16) *reinterpret_cast<uint4*>(crow + 16 * q) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+    }
+
+    // ---- every thread is done with this slot: refill it with the row nbuf steps ahead
     __syncthreads();
-    if (threadIdx.x < 32) {
-      const int lane = threadIdx.x;
-      float acc = 0.0f;
-      const int nchunk = K >> 3;
-      for (int c = lane; c < nchunk; c += 32) {
-        float t[8];
-        unpack_bf16x8(s_row[swz_chunk(c)], t);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc = __fmaf_rn(t[j], t[j], acc);
-      }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
-      if (lane == 0) {
-        const float mean = __fdiv_rn(acc, static_cast<float>(K));
-        const float var = __fadd_rn(mean, a.eps);
-        s_r = __fdiv_rn(1.0f, __fsqrt_rn(var));
+    if (tid == 0) {
+      const int64_t next = row + nbuf * stride;
+      if (next < a.rows) {
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&s_bar[slot], row_tx);
+        bulk_load(s_ring + slot * a.row_bytes, a.X + next * K, row_tx, &s_bar[slot]);
       }
     }
-    __syncthreads();
-    const float r = s_r;
-    const uint4* gr = reinterpret_cast<const uint4*>(a.gamma);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (8 * i < nel) {
-        float gm[8];
-        unpack_bf16x8(__ldg(gr + 8 * b + i), gm);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[8 * i + j] = __fmul_rn(__fmul_rn(v[8 * i + j], r), gm[j]);
-      }
-    }
-  }
-
-  if (do_wht && active) wht64(v);
-
-  // ---- amax: per 16-block and per row
-  float a16[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    float m = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[16 * q + i]));
-    a16[q] = m;
-  }
-  const float local = fmaxf(fmaxf(a16[0], a16[1]), fmaxf(a16[2], a16[3]));
-
-  if (MODE == kTensorAmax) {
-    const float A = block_max(local, s_red);
-    if (threadIdx.x == 0) atomicMax(a.amax_word, __float_as_uint(A));
-    return;
-  }
-  const float g = row_global<FMT, MODE>(a, local, s_red, row);
-  if (!active) return;
-
-  if (FMT == kNvfp4) {
-    const float six_g = __fmul_rn(6.0f, g);
-    const bool fast6g = rcp_ok(six_g);
-    const float r6g = fast6g ? rcp_approx(six_g) : 0.0f;
-    uint32_t sc_word = 0;
-    uint32_t cw[8];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint32_t sb8 =
-          (16 * q < nel) ? nvfp4_block(v + 16 * q, a16[q], g, six_g, r6g, fast6g, cw[2 * q], cw[2 * q + 1]) : 0u;
-      if (16 * q >= nel) cw[2 * q] = cw[2 * q + 1] = 0u;
-      sc_word |= sb8 << (8 * q);
-    }
-    uint4* crow = reinterpret_cast<uint4*>(a.codes + row * a.pitch + 32 * b);
-    crow[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-    crow[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-    store_scale_word(a.scales, row, b, nblk, sc_word);
-  } else {
-    const bool fast = rcp_ok(g);
-    const float r = fast ? rcp_approx(g) : 0.0f;
-    uint4* crow = reinterpret_cast<uint4*>(a.codes + row * a.pitch + 64 * b);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      if (16 * q < nel) {
-        uint32_t w[4];
-        fp8_block(v + 16 * q, g, r, fast, w);
-        crow[q] = make_uint4(w[0], w[1], w[2], w[3]);
-      }
+    if (++slot == nbuf) {
+      slot = 0;
+      phase ^= 1u;
     }
   }
 }
@@ -421,10 +402,30 @@ __global__ void finalize_global_kernel(float* g) {
   g[0] = __fdiv_rn(__uint_as_float(*reinterpret_cast<unsigned int*>(g)), 2688.0f);
 }
 
-inline int threads_for(int64_t K) {
-  const int64_t nblk = (K + 63) / 64;
-  const int64_t t = (nblk + 31) / 32 * 32;
-  return static_cast<int>(t < 32 ? 32 : t);
+template <int FMT, int MODE, bool NORM, bool WHT, int W>
+cudaError_t launch_ring(RowArgs a, cudaStream_t s) {
+  using C = RowCfg<W>;
+  auto kern = quant_rows_kernel<FMT, MODE, NORM, WHT, W>;
+  const int fit = C::kRingBytes / a.row_bytes;
+  a.nbuf = fit < 2 ? 2 : (fit > kMaxRowBufs ? kMaxRowBufs : fit);  // 2 x 64 KiB at the largest K
+  const size_t smem = static_cast<size_t>(a.nbuf) * a.row_bytes;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  // resident CTAs per SM: the register limit, or fewer where the rings do
+  // not fit (1 KiB per CTA is reserved by the SM)
+  int per_sm = static_cast<int>(228 * 1024 / (smem + 2048));
+  per_sm = per_sm < 1 ? 1 : (per_sm > C::kCtasPerSm ? C::kCtasPerSm : per_sm);
+  const int64_t ctas = static_cast<int64_t>(device_sm_count()) * per_sm;
+  const unsigned int grid = static_cast<unsigned int>(a.rows < ctas ? a.rows : ctas);
+  return launch_pdl(kern, dim3(grid), dim3(C::kThreads), smem, s, a);
+}
+
+template <int FMT, int MODE, bool NORM, bool WHT>
+cudaError_t launch_shape(const RowArgs& a, cudaStream_t s) {
+  if (a.K <= kShortRowK) return launch_ring<FMT, MODE, NORM, WHT, 8>(a, s);
+  return launch_ring<FMT, MODE, NORM, WHT, 16>(a, s);
 }
 
 template <int FMT, int MODE>
@@ -436,32 +437,21 @@ cudaError_t launch_rows(const void* X, int64_t rows, int64_t K, const void* gamm
   a.K = static_cast<int>(K);
   a.gamma = static_cast<const __nv_bfloat16*>(gamma);
   a.eps = eps;
-  a.flags = flags;
   a.codes = codes;
   a.pitch = pitch;
   a.scales = scales;
   a.gout = gout;
   a.amax_word = amax;
-  const bool norm = (MODE == kPerRow) && (flags & kFlagRmsNorm);
-  const bool xform = norm || (flags & kFlagHadamard);
-  const unsigned int grid = static_cast<unsigned int>(rows);
-  if (!xform) {
-    // one NVFP4 block per thread while a row fits in 512 threads
-    if (K <= 8192) {
-      const int threads = static_cast<int>(((K + 63) / 64 * 4 + 31) / 32 * 32);
-      return launch_pdl(quant_rows_plain_kernel<FMT, MODE, 16>, dim3(grid), dim3(threads), 0, s, a);
-    }
-    return launch_pdl(quant_rows_plain_kernel<FMT, MODE, 64>, dim3(grid), dim3(threads_for(K)), 0, s, a);
+  a.rows = rows;
+  a.nbuf = 0;
+  a.row_bytes = static_cast<int>((2 * K + 127) / 128 * 128);
+  a.budget = kWaitBudgetCycles;
+  const bool wht = (flags & kFlagHadamard) != 0;
+  if constexpr (MODE == kPerRow) {
+    if (flags & kFlagRmsNorm)
+      return wht ? launch_shape<FMT, MODE, true, true>(a, s) : launch_shape<FMT, MODE, true, false>(a, s);
   }
-  // staged bf16 row, rounded up to whole 64-element groups (the chunk
-  // swizzle permutes within groups of 8 chunks)
-  const size_t smem = norm ? static_cast<size_t>((K + 63) / 64) * 64 * 2 : 0;
-  auto kern = quant_rows_xform_kernel<FMT, MODE>;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-  }
-  return launch_pdl(kern, dim3(grid), dim3(threads_for(K)), smem, s, a);
+  return wht ? launch_shape<FMT, MODE, false, true>(a, s) : launch_shape<FMT, MODE, false, false>(a, s);
 }
 
 }  // namespace
@@ -491,6 +481,18 @@ cudaError_t launch_quant_weight_nvfp4(const void* W, int64_t N, int64_t K, uint3
 cudaError_t launch_quant_fp8(const void* X, int64_t rows, int64_t K, const void* gamma, float eps, uint32_t flags,
                              uint8_t* codes, float* s_out, cudaStream_t s) {
   return launch_rows<kFp8, kPerRow>(X, rows, K, gamma, eps, flags, codes, K, nullptr, s_out, nullptr, s);
+}
+
+cudaError_t read_and_clear_quant_status(unsigned int* out, cudaStream_t s) {
+  cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_vlaq_quant_status, sizeof(unsigned int), 0,
+                                            cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return e;
+  const unsigned int zero = 0;
+  e = cudaMemcpyToSymbolAsync(g_vlaq_quant_status, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return e;
+  return cudaStreamSynchronize(s);
 }
 
 }  // namespace vlaq
