@@ -74,7 +74,6 @@ struct GemmArgs {
   const __nv_bfloat16* residual;
   __nv_bfloat16* Y;
   float* partial;               // [splits][M][N] when splits > 1
-  unsigned int* counters;       // per output tile: splits finished (zeroed per call)
   int M, N, K;
   int k_steps;                  // MMA k-steps (64 fp4 or 32 fp8 elements each)
   int k_tiles;                  // stages of 4 k-steps
@@ -244,8 +243,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   const uint32_t tmem = s_tmem_base;
   // barrier setup, TMEM allocation and descriptor prefetch above overlap the
   // previous kernel's tail; global memory is touched only after this wait
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -446,67 +445,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 // The warpgroup register budgets add up to the launch allocation:
 // 128 + 168 + 168 + 48 = 4 x 128 per thread (the build checks that ptxas
 // allocates 128 registers at entry).
-// Last split of a tile: output = bf16(sum of the splits' fp32 partials, in
-// split order) * g_x[m] g_w + residual.  The tile's valid outputs are spread
-// over `nthreads` threads in 8-column groups; each group's partial loads are
-// issued four splits at a time so they overlap.
-__device__ __forceinline__ void splitk_finish_tile(const GemmArgs& a, int m_tile, int n_tile, int bn, int tid,
-                                                   int nthreads) {
-  const int r0 = m_tile * kBM, c0 = n_tile * bn;
-  const int rows = min(kBM, a.M - r0), cols = min(bn, a.N - c0);
-  const int groups = cols >> 3;  // N % 8 == 0
-  const size_t split_stride = static_cast<size_t>(a.M) * a.N;
-  for (int item = tid; item < rows * groups; item += nthreads) {
-    const int row = r0 + item / groups;
-    const int col = c0 + 8 * (item % groups);
-    const float* src = a.partial + static_cast<size_t>(row) * a.N + col;
-    float acc[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
-    int sp = 0;
-    for (; sp + 4 <= a.splits; sp += 4) {
-      float4 v[4][2];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const float4* p = reinterpret_cast<const float4*>(src + (sp + t) * split_stride);
-        v[t][0] = __ldcg(p);
-        v[t][1] = __ldcg(p + 1);
-      }
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        acc[0] += v[t][0].x; acc[1] += v[t][0].y; acc[2] += v[t][0].z; acc[3] += v[t][0].w;
-        acc[4] += v[t][1].x; acc[5] += v[t][1].y; acc[6] += v[t][1].z; acc[7] += v[t][1].w;
-      }
-    }
-    for (; sp < a.splits; ++sp) {
-      const float4* p = reinterpret_cast<const float4*>(src + sp * split_stride);
-      const float4 v0 = __ldcg(p), v1 = __ldcg(p + 1);
-      acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
-      acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
-    }
-    const float rs = a.xg[row] * a.wg[0];
-    float y[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) y[j] = acc[j] * rs;
-    const size_t o = static_cast<size_t>(row) * a.N + col;
-    if (a.residual) {
-      const uint4 rv = __ldg(reinterpret_cast<const uint4*>(a.residual + o));
-      const uint32_t wv[4] = {rv.x, rv.y, rv.z, rv.w};
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        y[2 * t] += __uint_as_float(wv[t] << 16);
-        y[2 * t + 1] += __uint_as_float(wv[t] & 0xFFFF0000u);
-      }
-    }
-    *reinterpret_cast<uint4*>(a.Y + o) = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
-                                                    pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
-  }
-}
-
-// Barrier over the eight epilogue warps (warps 4-11) of the scale-writer
-// kernel; id 0 is __syncthreads.
-__device__ __forceinline__ void epilogue_bar_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-
 struct SfwCfg {
   static constexpr int BN = 256;
   static constexpr int NRB = 2;
@@ -542,7 +480,6 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t s_tmem_base;
   __shared__ volatile int s_abort;
-  __shared__ int s_last;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
@@ -576,42 +513,75 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem_base;
-  // barrier setup, TMEM allocation and descriptor prefetch above overlap the
-  // previous kernel's tail; global memory is touched only after this wait
-  griddep_launch_dependents();
+
+  // Producer pieces of one pipeline stage: the weight half (B tile and its
+  // scales) and the activation half (A tile and its scales), both completing
+  // on the stage's full barrier armed with the bytes of both.
+  auto stage_bytes = [&](const Unit& w, int kt) -> uint32_t {
+    const int steps = min(4, args.k_steps - 4 * kt);
+    const int nrb = min(C::NRB, args.w_row_blocks - w.n * C::NRB);
+    return C::A_BYTES + C::B_BYTES + static_cast<uint32_t>(steps * 512 * (1 + nrb));
+  };
+  auto issue_weights = [&](int stage, const Unit& w, int kt) {
+    uint8_t* sb = smem + stage * C::STAGE_BYTES + C::A_BYTES;
+    uint8_t* ssfb = sb + C::B_BYTES + C::SFA_BYTES;
+    const int steps = min(4, args.k_steps - 4 * kt);
+    const int nrb = min(C::NRB, args.w_row_blocks - w.n * C::NRB);
+    tma_load_2d(sb, &tmB, &full_bar[stage], kt * 128, w.n * C::BN);
+    for (int rb = 0; rb < nrb; ++rb)
+      bulk_load(ssfb + rb * 2048, args.ws + (static_cast<size_t>(w.n * C::NRB + rb) * args.ka + 4 * kt) * 512,
+                steps * 512, &full_bar[stage]);
+  };
+  auto issue_acts = [&](int stage, const Unit& w, int kt) {
+    uint8_t* sa = smem + stage * C::STAGE_BYTES;
+    uint8_t* ssfa = sa + C::A_BYTES + C::B_BYTES;
+    const int steps = min(4, args.k_steps - 4 * kt);
+    tma_load_2d(sa, &tmA, &full_bar[stage], kt * 128, w.m * kBM);
+    bulk_load(ssfa, args.xs + (static_cast<size_t>(w.m) * args.ka + 4 * kt) * 512, steps * 512, &full_bar[stage]);
+  };
+
+  // Weights do not depend on the previous kernel on the stream (every
+  // library kernel triggers its dependents only after its own dependency
+  // wait, so all kernels two or more launches back, the weight quantizer
+  // among them, have completed): the first stages' weight halves stream in
+  // while the previous kernel (the activation quantizer) still runs.
+  int pre = 0;
+  uint32_t armed = 0;
+  if (warp == 0 && lane == 0) {
+    for (int u = blockIdx.x; u < args.units && pre < C::STAGES; u += gridDim.x) {
+      const Unit w = decode_unit(args, u);
+      for (int kt = w.kt0; kt < w.kt1 && pre < C::STAGES; ++kt, ++pre) {
+        mbar_arrive_expect_tx(&full_bar[pre], stage_bytes(w, kt));
+        armed |= 1u << pre;
+        issue_weights(pre, w, kt);
+      }
+    }
+  }
   griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t armed = 0, armed_phase = 0;
+      uint32_t armed_phase = 0;
+      int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
         const Unit w = decode_unit(args, u);
-        for (int kt = w.kt0; kt < w.kt1; ++kt) {
-          if (!wait_or_abort(&empty_bar[stage], phase ^ 1u, args.budget, &s_abort)) {
-            ok = false;
-            break;
+        for (int kt = w.kt0; kt < w.kt1; ++kt, ++it) {
+          if (it >= pre) {
+            if (!wait_or_abort(&empty_bar[stage], phase ^ 1u, args.budget, &s_abort)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full_bar[stage], stage_bytes(w, kt));
+            armed |= 1u << stage;
+            armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+            issue_weights(stage, w, kt);
           }
-          uint8_t* sa = smem + stage * C::STAGE_BYTES;
-          uint8_t* sb = sa + C::A_BYTES;
-          uint8_t* ssfa = sb + C::B_BYTES;
-          uint8_t* ssfb = ssfa + C::SFA_BYTES;
-          const int steps = min(4, args.k_steps - 4 * kt);
-          const int nrb = min(C::NRB, args.w_row_blocks - w.n * C::NRB);
-          mbar_arrive_expect_tx(&full_bar[stage],
-                                C::A_BYTES + C::B_BYTES + static_cast<uint32_t>(steps * 512 * (1 + nrb)));
-          armed |= 1u << stage;
-          armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
-          tma_load_2d(sa, &tmA, &full_bar[stage], kt * 128, w.m * kBM);
-          tma_load_2d(sb, &tmB, &full_bar[stage], kt * 128, w.n * C::BN);
-          bulk_load(ssfa, args.xs + (static_cast<size_t>(w.m) * args.ka + 4 * kt) * 512, steps * 512,
-                    &full_bar[stage]);
-          for (int rb = 0; rb < nrb; ++rb)
-            bulk_load(ssfb + rb * 2048, args.ws + (static_cast<size_t>(w.n * C::NRB + rb) * args.ka + 4 * kt) * 512,
-                      steps * 512, &full_bar[stage]);
+          issue_acts(stage, w, kt);
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -754,24 +724,12 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
         continue;
       }
-      // Split-K: store this split's fp32 partial sums; the split that
-      // finishes the tile last adds all partials in split order and writes
-      // the output (deterministic, no second kernel).
+      // Split-K: this split's fp32 partial sums; splitk_reduce_kernel adds
+      // the splits in order and applies the scales and the residual.
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int col0 = w.n * C::BN + 128 * h + 32 * c;
         if (row_ok && col0 < args.N) store_partial(args, w.split, row, col0, r[c]);
-      }
-      __threadfence();
-      epilogue_bar_sync();
-      if (e == 0 && lane == 0) {
-        const unsigned int done = atomicAdd(args.counters + (w.n * args.m_tiles + w.m), 1u);
-        s_last = (done == static_cast<unsigned int>(args.splits - 1));
-      }
-      epilogue_bar_sync();
-      if (s_last) {
-        __threadfence();
-        splitk_finish_tile(args, w.m, w.n, C::BN, e * 32 + lane, 256);
       }
     }
   }
@@ -792,8 +750,8 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int spli
                                      const float* __restrict__ xg, const float* __restrict__ wg,
                                      const __nv_bfloat16* __restrict__ residual,
                                      __nv_bfloat16* __restrict__ Y) {
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
   const int64_t idx8 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t total8 = static_cast<int64_t>(M) * N / 8;
   if (idx8 >= total8) return;
@@ -877,7 +835,6 @@ cudaError_t run(const uint8_t* xq, const uint8_t* xs, const float* xg, const uin
   a.residual = static_cast<const __nv_bfloat16*>(residual);
   a.Y = static_cast<__nv_bfloat16*>(Y);
   a.partial = static_cast<float*>(workspace);
-  a.counters = nullptr;
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.K = static_cast<int>(K);
@@ -893,16 +850,9 @@ cudaError_t run(const uint8_t* xq, const uint8_t* xs, const float* xg, const uin
   const int grid = plan.grid < a.units ? plan.grid : a.units;
   cudaError_t e;
   if (FP4 && BN == 256) {
-    if (plan.splits > 1) {
-      // tile counters live after the partial sums; they must start at zero
-      a.counters = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) + splitk_partial_bytes(plan.splits, M, N));
-      e = cudaMemsetAsync(a.counters, 0, sizeof(unsigned int) * static_cast<size_t>(a.m_tiles) * a.n_tiles, s);
-      if (e != cudaSuccess) return e;
-    }
     e = cudaFuncSetAttribute(gemm_fp4_sfw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SfwCfg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    // split-K partials are reduced inside the kernel
-    return launch_pdl(gemm_fp4_sfw_kernel, dim3(grid), dim3(SfwCfg::THREADS), SfwCfg::SMEM_BYTES, s, ta, tb, a);
+    e = launch_pdl(gemm_fp4_sfw_kernel, dim3(grid), dim3(SfwCfg::THREADS), SfwCfg::SMEM_BYTES, s, ta, tb, a);
   } else {
     auto kern = gemm_kernel<FP4, BN>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -927,8 +877,9 @@ GemmPlan plan_gemm(bool fp4, int64_t M, int64_t N, int64_t K, int num_sms) {
   const int64_t m_tiles = (M + kBM - 1) / kBM;
   if (fp4) {
     // NVFP4: always the 128 x 256 scale-writer kernel; few output tiles
-    // (decode) are split along K so every SM streams weights, and the last
-    // split of each tile reduces in-kernel.
+    // (decode) are split along K so every SM streams weights, and a second
+    // kernel adds the splits (no counters, so nothing has to be cleared
+    // between the activation quantizer and the GEMM).
     p.bn = 256;
     const int64_t tiles = m_tiles * ((N + 255) / 256);
     int64_t splits = 1;
@@ -940,7 +891,7 @@ GemmPlan plan_gemm(bool fp4, int64_t M, int64_t N, int64_t K, int num_sms) {
     p.splits = static_cast<int>(splits);
     const int64_t units = tiles * splits;
     p.grid = static_cast<int>(units < num_sms ? units : num_sms);
-    p.ws_bytes = splits > 1 ? splitk_partial_bytes(splits, M, N) + sizeof(unsigned int) * static_cast<size_t>(tiles) : 0;
+    p.ws_bytes = splits > 1 ? splitk_partial_bytes(splits, M, N) : 0;
     return p;
   }
   // Wide tiles halve the scale-factor copies per FLOP and the A re-reads;

@@ -10,9 +10,9 @@
 //
 // The array is a module global: every GPU that loads the library holds it
 // (kNoallocScratchBytes) until the process exits.  All calls on a device
-// share it and it keeps the last call's contents (each call clears, on its
-// stream, the tile counters that must start at zero); calls that overlap on the
-// GPU (different streams, or different host threads) race on it.
+// share it and it keeps the last call's contents (every partial sum is
+// written before it is read); calls that overlap on the GPU (different
+// streams, or different host threads) race on it.
 #include <cuda_runtime.h>
 
 #include <mutex>

@@ -67,6 +67,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // Lets the dependent grid start launching once every CTA of this grid has
 // executed this (or exited); the dependent still waits in griddep_wait().
+// Library kernels execute it only after their own griddep_wait(), so while
+// a library kernel runs, every kernel two or more launches back on the
+// stream has completed (the NVFP4 GEMM reads weights before its wait).
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }

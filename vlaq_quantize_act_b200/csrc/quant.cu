@@ -238,8 +238,8 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
     fence_mbarrier_init();
   }
   __syncthreads();
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
 
   if (tid == 0) {
     for (int b = 0; b < nbuf; ++b) {
@@ -397,8 +397,8 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
 }
 
 __global__ void finalize_global_kernel(float* g) {
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
   g[0] = __fdiv_rn(__uint_as_float(*reinterpret_cast<unsigned int*>(g)), 2688.0f);
 }
 
