@@ -494,11 +494,11 @@ def main():
                    "l2": "inputs larger than L2 (per-step working set ~294 MB)", "graph": True},
         "roofline": {"bound": "tensor", "achieved": g_ach, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": g_ach / fp4_peak, "traffic": traffic,
-                     "kernel": "gemm_kernel<FP4> gate_up 1024x37888x3584 (2MNK = 278.1 GFLOP per launch)",
+                     "kernel": "gemm_fp4_sfw_kernel gate_up 1024x37888x3584 (2MNK = 278.1 GFLOP per launch)",
                      "all_gemms_tflops": gemm_all, "timing": f"CUDA events in a {tmode} capture of the step",
                      "peak_note": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 4 (nominal FP4:BF16)"},
         "prologue": {"bound": "hbm", "achieved": p_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": p_ach / peaks["hbm_gbs"], "kernel": "quant_rows_kernel<NVFP4>"},
+                     "frac": p_ach / peaks["hbm_gbs"], "kernel": "quant_rows_kernel (NVFP4 activation prologue)"},
         "per_projection": per_proj,
         "clocks": clocks,
     }
