@@ -151,8 +151,13 @@ VLAQ_API vlaq_status vlaq_quantize_act_nvfp4(const void* X, int64_t M, int64_t K
 
 /* Bytes of workspace vlaq_linear_nvfp4 / vlaq_linear_fp8 need for the given
  * shape on the current device (0 when the shape runs without split-K).  The
- * workspace holds per-split fp32 partial sums; its contents on entry do not
- * matter (every partial sum is written before a second kernel adds them). */
+ * workspace's first 1024 bytes hold vlaq_linear_nvfp4's per-tile arrival
+ * counters, the per-split fp32 partial sums follow.  The counters must be
+ * zero when a call starts: zero the workspace once after allocating it;
+ * every call (of any shape, NVFP4 or FP8) leaves them zero again, so nothing
+ * is cleared between calls.  After vlaq_check reports VLAQ_ERR_TIMEOUT, zero
+ * the workspace again before reusing it.  Calls that share a workspace
+ * must not overlap on the GPU. */
 VLAQ_API size_t vlaq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* Y = bf16_rne( (sum_k dec(x)[m,k] * dec(w)[n,k]) + residual[m,n] )
@@ -184,10 +189,10 @@ VLAQ_API vlaq_status vlaq_linear_nvfp4(const uint8_t* xq, const uint8_t* xs,
  * with VLAQ_ERR_WORKSPACE (use vlaq_linear_nvfp4 then).  The first call on
  * each device looks the array's address up (cudaGetSymbolAddress) and caches
  * it; make that first call before any stream capture.  All calls on a
- * device share the array and it keeps the last call's contents (every
- * partial sum is written before it is read, so nothing is cleared);
- * calls that overlap on the GPU, e.g. on two streams, race on it and must
- * be serialized by the caller.  The source pages have no counterpart of
+ * device share the array (zero when the library loads; each call leaves its
+ * tile counters zero again, and vlaq_check clears the array when it
+ * reports VLAQ_ERR_TIMEOUT); calls that overlap on the GPU, e.g. on two
+ * streams, race on it and must be serialized by the caller.  The source pages have no counterpart of
  * this entry point. */
 VLAQ_API vlaq_status vlaq_linear_nvfp4_noalloc(const uint8_t* xq, const uint8_t* xs,
                                       const float* g_x, const uint8_t* wq,

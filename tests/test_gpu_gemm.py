@@ -163,3 +163,34 @@ def test_linear_fp8_wide_tiles_vs_oracle(M, N, K, res):
     Y = gpu_linear_fp8(to_dev(cx), to_dev(sx), to_dev(cw), to_dev(sw), M, N, K, None if R is None else R.cuda())
     rel, mx = gemm_error(Y, Y64)
     assert rel < REL_FRO_TOL, (rel, mx)
+
+
+def test_split_workspace_reused_across_calls_and_shapes():
+    """The NVFP4 split-K tile counters return to zero after every call: one
+    zeroed workspace serves repeated calls and shapes with different split
+    counts.  A counter left non-zero would keep the next call's last split
+    from recognising itself, and its tile would stay NaN."""
+    m = vq()
+    shapes = [(1, 512, 4096), (4, 1024, 3584), (8, 256, 2048)]
+    need = max(m.vlaq_linear_workspace_bytes(*s) for s in shapes)
+    assert all(m.vlaq_linear_workspace_bytes(*s) > 0 for s in shapes)  # all three split K
+    wsp = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    cases = {s: _oracle_case(*s, 51) for s in shapes}
+    dev = {}
+    for (M, N, K), (cx, sx, gx, cw, sw, gw, _, _) in cases.items():
+        dev[(M, N, K)] = (to_dev(layouts.pad_codes(cx, K)), to_dev(layouts.tile_scales(sx, M, K)), to_dev(gx),
+                          to_dev(layouts.pad_codes(cw, K)), to_dev(layouts.tile_scales(sw, N, K)), to_dev(gw))
+    first = {}
+    for rep in range(3):
+        for (M, N, K) in shapes:
+            Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+            m.vlaq_linear_nvfp4(*dev[(M, N, K)], None, Y, M, N, K, wsp, need)
+            torch.cuda.synchronize()
+            m.vlaq_check()
+            y = Y.float().cpu().numpy()
+            rel, mx = gemm_error(y, cases[(M, N, K)][-1])
+            assert rel < REL_FRO_TOL, (rep, M, N, K, rel, mx)
+            if rep == 0:
+                first[(M, N, K)] = y
+            else:
+                assert np.array_equal(y, first[(M, N, K)]), (rep, M, N, K)

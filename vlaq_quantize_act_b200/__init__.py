@@ -176,8 +176,10 @@ def alloc_fp8(rows: int, K: int, device="cuda"):
 
 
 def alloc_workspace(M: int, N: int, K: int, device="cuda"):
-    """(workspace tensor or None, bytes) for vlaq_linear_*."""
+    """(workspace tensor or None, bytes) for vlaq_linear_*, allocated zeroed:
+    the NVFP4 split-K tile counters must start at zero (every call leaves
+    them zero again)."""
     n = vlaq_linear_workspace_bytes(M, N, K)
     if n == 0:
         return None, 0
-    return torch.empty((n + 15) // 16 * 16, dtype=torch.uint8, device=device), n
+    return torch.zeros((n + 15) // 16 * 16, dtype=torch.uint8, device=device), n

@@ -120,8 +120,14 @@ vlaq_status vlaq_check(void* stream) {
   e = vlaq::read_and_clear_quant_status(&qst, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail("vlaq_check", e);
   st |= qst;
-  if (st & vlaq::kStatusTimeout)
-    return fail(VLAQ_ERR_TIMEOUT, "vlaq_check: a kernel gave up a bounded wait (device status 0x%x)", st);
+  if (st & vlaq::kStatusTimeout) {
+    // a GEMM that gave up may have left split-K tile counters non-zero
+    e = vlaq::noalloc_clear(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail("vlaq_check", e);
+    return fail(VLAQ_ERR_TIMEOUT,
+                "vlaq_check: a kernel gave up a bounded wait (device status 0x%x); zero any split-K workspace "
+                "before reusing it", st);
+  }
   return ok();
 }
 

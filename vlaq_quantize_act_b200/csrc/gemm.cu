@@ -75,6 +75,7 @@ struct GemmArgs {
   __nv_bfloat16* Y;
   float* partial;               // [splits][M][N] when splits > 1
   int M, N, K;
+  unsigned int* counters;       // per output tile: splits arrived (zero between calls)
   int k_steps;                  // MMA k-steps (64 fp4 or 32 fp8 elements each)
   int k_tiles;                  // stages of 4 k-steps
   int m_tiles, n_tiles, splits;
@@ -445,6 +446,67 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 // The warpgroup register budgets add up to the launch allocation:
 // 128 + 168 + 168 + 48 = 4 x 128 per thread (the build checks that ptxas
 // allocates 128 registers at entry).
+// Last split of a tile: output = bf16(sum of the splits' fp32 partials, in
+// split order) * g_x[m] g_w + residual.  The tile's valid outputs are spread
+// over `nthreads` threads in 8-column groups; each group's partial loads are
+// issued four splits at a time so they overlap.
+__device__ __forceinline__ void splitk_finish_tile(const GemmArgs& a, int m_tile, int n_tile, int bn, int tid,
+                                                   int nthreads) {
+  const int r0 = m_tile * kBM, c0 = n_tile * bn;
+  const int rows = min(kBM, a.M - r0), cols = min(bn, a.N - c0);
+  const int groups = cols >> 3;  // N % 8 == 0
+  const size_t split_stride = static_cast<size_t>(a.M) * a.N;
+  for (int item = tid; item < rows * groups; item += nthreads) {
+    const int row = r0 + item / groups;
+    const int col = c0 + 8 * (item % groups);
+    const float* src = a.partial + static_cast<size_t>(row) * a.N + col;
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+    int sp = 0;
+    for (; sp + 4 <= a.splits; sp += 4) {
+      float4 v[4][2];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float4* p = reinterpret_cast<const float4*>(src + (sp + t) * split_stride);
+        v[t][0] = __ldcg(p);
+        v[t][1] = __ldcg(p + 1);
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        acc[0] += v[t][0].x; acc[1] += v[t][0].y; acc[2] += v[t][0].z; acc[3] += v[t][0].w;
+        acc[4] += v[t][1].x; acc[5] += v[t][1].y; acc[6] += v[t][1].z; acc[7] += v[t][1].w;
+      }
+    }
+    for (; sp < a.splits; ++sp) {
+      const float4* p = reinterpret_cast<const float4*>(src + sp * split_stride);
+      const float4 v0 = __ldcg(p), v1 = __ldcg(p + 1);
+      acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
+      acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
+    }
+    const float rs = a.xg[row] * a.wg[0];
+    float y[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = acc[j] * rs;
+    const size_t o = static_cast<size_t>(row) * a.N + col;
+    if (a.residual) {
+      const uint4 rv = __ldg(reinterpret_cast<const uint4*>(a.residual + o));
+      const uint32_t wv[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        y[2 * t] += __uint_as_float(wv[t] << 16);
+        y[2 * t + 1] += __uint_as_float(wv[t] & 0xFFFF0000u);
+      }
+    }
+    *reinterpret_cast<uint4*>(a.Y + o) = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
+                                                    pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+  }
+}
+
+// Barrier over the eight epilogue warps (warps 4-11) of the scale-writer
+// kernel; id 0 is __syncthreads.
+__device__ __forceinline__ void epilogue_bar_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
 struct SfwCfg {
   static constexpr int BN = 256;
   static constexpr int NRB = 2;
@@ -480,6 +542,7 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t s_tmem_base;
   __shared__ volatile int s_abort;
+  __shared__ int s_last;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
@@ -724,12 +787,30 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
         continue;
       }
-      // Split-K: this split's fp32 partial sums; splitk_reduce_kernel adds
-      // the splits in order and applies the scales and the residual.
+      // Split-K: store this split's fp32 partial sums; the split that
+      // arrives last at the tile's counter adds all partials in split order
+      // and writes the output (deterministic, no second kernel), and puts
+      // the counter back to zero for the next call.  Nothing clears the
+      // counters between calls: the next GEMM on the stream reaches its
+      // epilogue only after this grid has completed (every library kernel
+      // triggers its dependents after its own dependency wait).
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int col0 = w.n * C::BN + 128 * h + 32 * c;
         if (row_ok && col0 < args.N) store_partial(args, w.split, row, col0, r[c]);
+      }
+      __threadfence();
+      epilogue_bar_sync();
+      if (e == 0 && lane == 0) {
+        unsigned int* cnt = args.counters + (w.n * args.m_tiles + w.m);
+        const unsigned int done = atomicAdd(cnt, 1u);
+        s_last = (done == static_cast<unsigned int>(args.splits - 1));
+        if (s_last) *cnt = 0u;  // every split of this call has arrived
+      }
+      epilogue_bar_sync();
+      if (s_last) {
+        __threadfence();
+        splitk_finish_tile(args, w.m, w.n, C::BN, e * 32 + lane, 256);
       }
     }
   }
@@ -834,7 +915,9 @@ cudaError_t run(const uint8_t* xq, const uint8_t* xs, const float* xg, const uin
   a.wg = wg;
   a.residual = static_cast<const __nv_bfloat16*>(residual);
   a.Y = static_cast<__nv_bfloat16*>(Y);
-  a.partial = static_cast<float*>(workspace);
+  a.partial = plan.splits > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kSplitCounterBytes)
+                              : nullptr;
+  a.counters = nullptr;
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.K = static_cast<int>(K);
@@ -850,9 +933,12 @@ cudaError_t run(const uint8_t* xq, const uint8_t* xs, const float* xg, const uin
   const int grid = plan.grid < a.units ? plan.grid : a.units;
   cudaError_t e;
   if (FP4 && BN == 256) {
+    // tile counters: the first bytes of the workspace (zero between calls)
+    if (plan.splits > 1) a.counters = static_cast<unsigned int*>(workspace);
     e = cudaFuncSetAttribute(gemm_fp4_sfw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SfwCfg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(gemm_fp4_sfw_kernel, dim3(grid), dim3(SfwCfg::THREADS), SfwCfg::SMEM_BYTES, s, ta, tb, a);
+    // split-K partials are reduced inside the kernel
+    return launch_pdl(gemm_fp4_sfw_kernel, dim3(grid), dim3(SfwCfg::THREADS), SfwCfg::SMEM_BYTES, s, ta, tb, a);
   } else {
     auto kern = gemm_kernel<FP4, BN>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -864,7 +950,7 @@ cudaError_t run(const uint8_t* xq, const uint8_t* xs, const float* xg, const uin
   const int threads = 256;
   const int64_t blocks = (total8 + threads - 1) / threads;
   return launch_pdl(splitk_reduce_kernel<FP4>, dim3(static_cast<unsigned int>(blocks)), dim3(threads), 0, s,
-                    static_cast<const float*>(workspace), plan.splits, a.M, a.N, xg, wg,
+                    static_cast<const float*>(a.partial), plan.splits, a.M, a.N, xg, wg,
                     static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(Y));
 }
 
@@ -877,13 +963,13 @@ GemmPlan plan_gemm(bool fp4, int64_t M, int64_t N, int64_t K, int num_sms) {
   const int64_t m_tiles = (M + kBM - 1) / kBM;
   if (fp4) {
     // NVFP4: always the 128 x 256 scale-writer kernel; few output tiles
-    // (decode) are split along K so every SM streams weights, and a second
-    // kernel adds the splits (no counters, so nothing has to be cleared
-    // between the activation quantizer and the GEMM).
+    // (decode) are split along K so every SM streams weights, and the last
+    // split of each tile reduces in-kernel (per-tile counters after the
+    // partials, zero between calls).
     p.bn = 256;
     const int64_t tiles = m_tiles * ((N + 255) / 256);
     int64_t splits = 1;
-    if (tiles * 2 <= num_sms) {
+    if (tiles * 2 <= num_sms && tiles * sizeof(unsigned int) <= kSplitCounterBytes) {
       splits = num_sms / tiles;
       if (splits > k_tiles) splits = k_tiles;
       if (splits < 1) splits = 1;
@@ -891,7 +977,7 @@ GemmPlan plan_gemm(bool fp4, int64_t M, int64_t N, int64_t K, int num_sms) {
     p.splits = static_cast<int>(splits);
     const int64_t units = tiles * splits;
     p.grid = static_cast<int>(units < num_sms ? units : num_sms);
-    p.ws_bytes = splits > 1 ? splitk_partial_bytes(splits, M, N) : 0;
+    p.ws_bytes = splits > 1 ? kSplitCounterBytes + splitk_partial_bytes(splits, M, N) : 0;
     return p;
   }
   // Wide tiles halve the scale-factor copies per FLOP and the A re-reads;
@@ -916,7 +1002,7 @@ GemmPlan plan_gemm(bool fp4, int64_t M, int64_t N, int64_t K, int num_sms) {
   p.splits = static_cast<int>(splits);
   const int64_t units = tiles * splits;
   p.grid = static_cast<int>(units < num_sms ? units : num_sms);
-  p.ws_bytes = splits > 1 ? static_cast<size_t>(splits) * M * N * sizeof(float) : 0;
+  p.ws_bytes = splits > 1 ? kSplitCounterBytes + splitk_partial_bytes(splits, M, N) : 0;
   return p;
 }
 

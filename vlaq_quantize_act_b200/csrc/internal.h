@@ -43,6 +43,11 @@ struct GemmPlan {
   size_t ws_bytes; // fp32 partials needed when splits > 1
 };
 GemmPlan plan_gemm(bool fp4, int64_t M, int64_t N, int64_t K, int num_sms);
+// Split-K workspace layout: the NVFP4 per-tile arrival counters occupy the
+// first kSplitCounterBytes (zero between calls, the same place for every
+// shape, so no shape's partial sums ever overwrite them), the fp32 partial
+// sums follow.  Split plans have at most num_sms / 2 tiles.
+constexpr size_t kSplitCounterBytes = 1024;
 // fp32 partial sums of a split-K plan, rounded up to 256 bytes.
 inline size_t splitk_partial_bytes(int64_t splits, int64_t M, int64_t N) {
   return (static_cast<size_t>(splits) * M * N * sizeof(float) + 255) / 256 * 256;
@@ -84,5 +89,6 @@ int device_sm_count();
 constexpr size_t kNoallocScratchBytes = size_t(4) << 20;  // 4 MiB per device
 constexpr int kMaxDevices = 64;
 cudaError_t noalloc_scratch(void** out);
+cudaError_t noalloc_clear(cudaStream_t s);
 
 }  // namespace vlaq

@@ -10,9 +10,10 @@
 //
 // The array is a module global: every GPU that loads the library holds it
 // (kNoallocScratchBytes) until the process exits.  All calls on a device
-// share it and it keeps the last call's contents (every partial sum is
-// written before it is read); calls that overlap on the GPU (different
-// streams, or different host threads) race on it.
+// share it.  It is zero when the module loads and the GEMM leaves its
+// split-K tile counters zero after every call; after a timed-out call
+// vlaq_check clears it (noalloc_clear).  Calls that overlap on the GPU
+// (different streams, or different host threads) race on it.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -45,6 +46,21 @@ cudaError_t noalloc_scratch(void** out) {
   }
   *out = g_ptr[dev];
   return cudaSuccess;
+}
+
+// Zeroes the scratch array of the current device on stream s (only if a
+// call has resolved it on this device).
+cudaError_t noalloc_clear(cudaStream_t s) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaSuccess;
+  void* p = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    p = g_ptr[dev];
+  }
+  return p ? cudaMemsetAsync(p, 0, kNoallocScratchBytes, s) : cudaSuccess;
 }
 
 }  // namespace vlaq
