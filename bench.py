@@ -426,7 +426,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="vlaq", choices=["vlaq", "reference"])
     ap.add_argument("--ref-rows", type=int, default=4)
-    ap.add_argument("--cpu-rows", type=int, default=16)
+    ap.add_argument("--cpu-rows", type=int, default=768)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the decode / fp8 / e2e extras")
     args = ap.parse_args()

@@ -38,7 +38,8 @@ def _run_nvfp4_from_oracle(M, N, K, case):
 
 
 # (M, N, K): one tile; ragged M / N / K tails; several K stages; split-K
-# decode shapes (M <= 8 with few N tiles); residual add.
+# decode shapes (M <= 8 with few N tiles); residual add; the last row count
+# of the few-row kernel (32) and the first of the wide one (33).
 NVFP4_CASES = [
     (16, 128, 256, False),
     (128, 128, 256, False),
@@ -50,6 +51,8 @@ NVFP4_CASES = [
     (8, 1024, 3584, False),
     (1, 8, 64, False),
     (64, 4608, 256, False),
+    (32, 264, 512, True),
+    (33, 256, 1024, False),
 ]
 
 
