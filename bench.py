@@ -139,6 +139,9 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ setup
+RANK_SEED_STRIDE = 1000  # activation seed offset per rank
+
+
 def make_inputs(M, device, seed_offset=0):
     data = {}
     for name in PROJ:
@@ -452,7 +455,9 @@ def main():
 
     peaks = load_peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
-    data = make_inputs(M_PREFILL, "cpu", seed_offset=0)
+    # weak scaling: every rank quantizes and multiplies its own tokens (its
+    # own activation seeds) against the same weights
+    data = make_inputs(M_PREFILL, "cpu", seed_offset=RANK_SEED_STRIDE * rank)
 
     # ---------------- prefill NVFP4 step (graph replays)
     step = Step(vq, data, M_PREFILL, device)
