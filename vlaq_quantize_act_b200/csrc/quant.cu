@@ -273,12 +273,19 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
     float r = 1.0f;
     if (NORM) {
       if (warp == 0) {
+        // the chain of fused multiply-adds is fixed; the next chunk's load
+        // is issued before the current chunk's eight steps
+        const uint4* rs4 = reinterpret_cast<const uint4*>(rs);
+        const int nch = K >> 3;
         float acc = 0.0f;
-        for (int c = lane; c < (K >> 3); c += 32) {
+        uint4 cur = lane < nch ? rs4[lane] : make_uint4(0, 0, 0, 0);
+        for (int c = lane; c < nch; c += 32) {
+          const uint4 nxt = c + 32 < nch ? rs4[c + 32] : make_uint4(0, 0, 0, 0);
           float t[8];
-          unpack_bf16x8(reinterpret_cast<const uint4*>(rs)[c], t);
+          unpack_bf16x8(cur, t);
 #pragma unroll
           for (int j = 0; j < 8; ++j) acc = __fmaf_rn(t[j], t[j], acc);
+          cur = nxt;
         }
 #pragma unroll
         for (int o = 16; o; o >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
