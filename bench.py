@@ -222,6 +222,55 @@ class Step:
         return M * K * 2 + M * K // 2 + M * K // 16 + 4 * M
 
 
+def stack_weights(vq, device, layers=si.STACK_LAYERS):
+    """NVFP4 weights of the 28-layer stack in (layer, projection) order, each
+    quantized on the device right after it is generated (only the NVFP4 copy
+    stays: about 3.7 GB)."""
+    out = []
+    for l in range(layers):
+        for p, (name, K, N) in enumerate(si.STACK_PROJECTIONS):
+            W = si.projection_weight(K, N, si.stack_seed(l, p)).to(device)
+            wq, ws, wg = vq.alloc_nvfp4(N, K, device, per_tensor=True)
+            vq.vlaq_quantize_weight_nvfp4(W, N, K, 0, wq, ws, wg)
+            del W
+            out.append((wq, ws, wg))
+    torch.cuda.synchronize()
+    return out
+
+
+class Stack:
+    """The 28-layer stack of seven unfused projections (196 NVFP4 GEMMs):
+    every (layer, projection) has its own seeded weight and its own seeded
+    activations [M, K]; run() is one prologue + GEMM per entry."""
+
+    def __init__(self, vq, M, device, layers=si.STACK_LAYERS, weights=None):
+        self.vq = vq
+        self.M = M
+        self.entries = []
+        if weights is None:
+            weights = stack_weights(vq, device, layers)
+        for l in range(layers):
+            for p, (name, K, N) in enumerate(si.STACK_PROJECTIONS):
+                seed = si.stack_seed(l, p)
+                wq, ws, wg = weights[7 * l + p]
+                X = si.projection_activations(K, M, seed).to(device)
+                wsp, nb = vq.alloc_workspace(M, N, K, device)
+                self.entries.append(dict(layer=l, proj=p, name=name, K=K, N=N, W=(wq, ws, wg), X=X,
+                                         act=vq.alloc_nvfp4(M, K, device),
+                                         Y=torch.empty(M, N, dtype=torch.bfloat16, device=device), ws=wsp, nb=nb))
+        torch.cuda.synchronize()
+        self.flops = sum(2.0 * M * e["N"] * e["K"] for e in self.entries)
+        self.weight_bytes = sum(e["W"][0].numel() + e["W"][1].numel() + 4 for e in self.entries)
+
+    def run(self, copy=0):
+        vq, M = self.vq, self.M
+        for e in self.entries:
+            xq, xs, xg = e["act"]
+            wq, ws, wg = e["W"]
+            vq.vlaq_quantize_act_nvfp4(e["X"], M, e["K"], None, 1e-6, 0, xq, xs, xg)
+            vq.vlaq_linear_nvfp4(xq, xs, xg, wq, ws, wg, None, e["Y"], M, e["N"], e["K"], e["ws"], e["nb"])
+
+
 def capture(step, copies=1):
     """CUDA graph of `copies` consecutive steps (rotating weight copies)."""
     s = torch.cuda.Stream()
@@ -432,6 +481,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=768)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the decode / fp8 / e2e extras")
+    ap.add_argument("--stack", action="store_true",
+                    help="also time the 28-layer stack (196 GEMMs) at M = 1024 and M = 1 (about a minute of setup)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -570,6 +621,26 @@ def main():
         ems = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist_on, device)
         out["e2e"] = {"value": world * step.flops / (ems / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ems,
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if args.stack:
+        # ---------------- 28-layer stack: one graph of 196 prologue + GEMM pairs
+        out["stack"] = {}
+        sw = stack_weights(vq, device)
+        for sm in (M_PREFILL, 1):
+            st = Stack(vq, sm, device, weights=sw)
+            sg = capture(st)
+            for _ in range(args.warmup):
+                sg.replay()
+            torch.cuda.synchronize()
+            sms = time_graph(sg, max(args.steps // 4, 3), dist_on, device)
+            key = "prefill" if sm > 1 else "decode"
+            out["stack"][key] = {"M": sm, "ms": sms, "us_per_token": 1e3 * sms / sm,
+                                 "tflops": world * st.flops / (sms / 1e3) / 1e12,
+                                 "weight_gbs": world * st.weight_bytes / (sms / 1e3) / 1e9,
+                                 "gemms": len(st.entries)}
+            del sg, st
+            torch.cuda.empty_cache()
+        del sw
 
     # launches of our kernels inside the timed region: per step 4 prologues +
     # 4 GEMMs (+ split-K reductions when planned)
