@@ -149,6 +149,18 @@ VLAQ_API vlaq_status vlaq_quantize_act_nvfp4(const void* X, int64_t M, int64_t K
                                     uint8_t* scales, float* g_x,
                                     void* stream);
 
+/* Block scales from the 128x4 tiled layout the GEMM reads (as written by
+ * the NVFP4 quantizers, vlaq_nvfp4_scale_bytes(rows, K) bytes) to the
+ * logical row-major layout: out[r * (K/16) + b] = E4M3 scale of row r,
+ * 16-block b, for r < rows, b < K/16 (padding rows and columns dropped).
+ *   in   device, 16-byte aligned;  out  device, rows * K/16 bytes
+ * K % 16 != 0 is refused with the division in the message.  The layout
+ * change itself is this library's: the pages store scales row-major
+ * ("NVFP4 block scale per 16 values", [Recipes] NVFP4 loader commit), the
+ * tensor cores read the tiled layout. */
+VLAQ_API vlaq_status vlaq_scales_to_rowmajor(const uint8_t* in, uint8_t* out, int64_t rows, int64_t K,
+                                             void* stream);
+
 /* Bytes of workspace vlaq_linear_nvfp4 / vlaq_linear_fp8 need for the given
  * shape on the current device (0 when the shape runs without split-K).  The
  * workspace's first 1024 bytes hold vlaq_linear_nvfp4's per-tile arrival

@@ -132,3 +132,9 @@ def test_no_device_is_an_error_not_a_fallback(vq):
     with pytest.raises(vq.VlaqError) as ei:
         vq.vlaq_quantize_act_nvfp4(FAKE, 4, 256, None, 1e-6, 0, FAKE, FAKE, FAKE)
     assert ei.value.status in (4, 5)
+
+
+def test_scales_to_rowmajor_refuses_bad_k(vq):
+    with pytest.raises(vq.VlaqError) as ei:
+        vq._check(vq._lib.vlaq_scales_to_rowmajor(16, 16, 4, 3420, None))
+    assert ei.value.status == 2 and "3420 / 16 = 213.75" in ei.value.message

@@ -6,8 +6,9 @@ import torch
 
 import oracle
 import synthetic_inputs as si
+import layouts
 from gpu_helpers import (assert_nvfp4_equal, bits, gpu_quant_act_nvfp4, gpu_quant_fp8,
-                         gpu_quant_weight_nvfp4)
+                         gpu_quant_weight_nvfp4, to_dev, vq)
 
 pytestmark = pytest.mark.gpu
 
@@ -140,3 +141,33 @@ def test_act_nvfp4_values_near_decision_points():
         Xs = (X.float() * scale).to(torch.bfloat16)
         ref = oracle.quantize_nvfp4(bits(Xs))
         assert_nvfp4_equal(gpu_quant_act_nvfp4(Xs), ref, Xs.shape[0], 64, f"near points x{scale}")
+
+
+@pytest.mark.parametrize("M,K", [(300, 1008), (1, 3584), (129, 16), (1024, 18944)])
+def test_scales_to_rowmajor_matches_oracle(M, K):
+    """GPU quantizer's tiled scales, converted back to the logical row-major
+    layout by vlaq_scales_to_rowmajor, equal the oracle's scales byte for
+    byte (K / 16 = 63 and 1 exercise the partial last word of a row)."""
+    m = vq()
+    X = si.projection_activations(K, M, 61)
+    xq, xs, xg = m.alloc_nvfp4(M, K)
+    m.vlaq_quantize_act_nvfp4(X.cuda(), M, K, None, 1e-6, 0, xq, xs, xg)
+    out = torch.full((M, K // 16), 0xAB, dtype=torch.uint8, device="cuda")
+    m.vlaq_scales_to_rowmajor(xs, out, M, K)
+    torch.cuda.synchronize()
+    m.vlaq_check()
+    _, sref, _ = oracle.quantize_nvfp4(bits(X))
+    assert np.array_equal(out.cpu().numpy(), sref)
+
+
+def test_scales_to_rowmajor_random_buffer():
+    """Any tiled buffer: the conversion equals the layout's definition
+    (test-side index math), padding dropped."""
+    m = vq()
+    rows, K = 257, 336
+    n = layouts.scale_bytes(rows, K)
+    buf = np.random.default_rng(3).integers(0, 256, n, dtype=np.uint8)
+    out = torch.empty(rows, K // 16, dtype=torch.uint8, device="cuda")
+    m.vlaq_scales_to_rowmajor(to_dev(buf), out, rows, K)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy(), layouts.untile_scales(buf, rows, K))

@@ -60,6 +60,7 @@ _SIGS = {
     "vlaq_quantize_act_fp8": (ctypes.c_int, [_P, _I64, _I64, _P, _F, _U32, _P, _P, _P]),
     "vlaq_linear_fp8": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "vlaq_linear_nvfp4_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "vlaq_scales_to_rowmajor": (ctypes.c_int, [_P, _P, _I64, _I64, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -129,6 +130,10 @@ def vlaq_quantize_weight_nvfp4(W, N, K, flags, codes, scales, g_w, stream=None):
 def vlaq_quantize_act_nvfp4(X, M, K, gamma, eps, flags, codes, scales, g_x, stream=None):
     _check(_lib.vlaq_quantize_act_nvfp4(_ptr(X), M, K, _ptr(gamma), eps, flags, _ptr(codes), _ptr(scales),
                                         _ptr(g_x), _stream(stream)))
+
+
+def vlaq_scales_to_rowmajor(scales, out, rows, K, stream=None):
+    _check(_lib.vlaq_scales_to_rowmajor(_ptr(scales), _ptr(out), rows, K, _stream(stream)))
 
 
 def vlaq_linear_nvfp4(xq, xs, g_x, wq, ws, g_w, residual, Y, M, N, K, workspace=None, ws_bytes=0,

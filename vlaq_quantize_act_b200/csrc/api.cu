@@ -170,6 +170,21 @@ vlaq_status vlaq_quantize_weight_nvfp4(const void* W, int64_t N, int64_t K, uint
   return ok();
 }
 
+vlaq_status vlaq_scales_to_rowmajor(const uint8_t* in, uint8_t* out, int64_t rows, int64_t K, void* stream) {
+  const char* fn = "vlaq_scales_to_rowmajor";
+  vlaq_status st;
+  if ((st = check_k(fn, K, 0, true, 0))) return st;
+  if (rows < 0) return fail(VLAQ_ERR_INVALID_ARG, "%s: rows = %lld is negative", fn, (long long)rows);
+  if (rows > 0x7FFFFFFF) return fail(VLAQ_ERR_SHAPE, "%s: rows = %lld is too large", fn, (long long)rows);
+  if (rows == 0) return ok();
+  VLAQ_NONNULL(fn, in);
+  if (!out) return fail(VLAQ_ERR_INVALID_ARG, "%s: out is NULL", fn);
+  if ((st = check_device(fn))) return st;
+  cudaError_t e = vlaq::launch_scales_to_rowmajor(in, out, rows, K, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(fn, e);
+  return ok();
+}
+
 vlaq_status vlaq_quantize_weight_fp8(const void* W, int64_t N, int64_t K, uint32_t flags, uint8_t* codes,
                                      float* s_w, void* stream) {
   const char* fn = "vlaq_quantize_weight_fp8";

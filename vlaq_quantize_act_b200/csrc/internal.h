@@ -34,6 +34,7 @@ cudaError_t launch_quant_weight_nvfp4(const void* W, int64_t N, int64_t K, uint3
                                       uint8_t* codes, uint8_t* scales, float* g_w, cudaStream_t s);
 cudaError_t launch_quant_fp8(const void* X, int64_t rows, int64_t K, const void* gamma, float eps,
                              uint32_t flags, uint8_t* codes, float* s_out, cudaStream_t s);
+cudaError_t launch_scales_to_rowmajor(const uint8_t* in, uint8_t* out, int64_t rows, int64_t K, cudaStream_t s);
 
 // ---- GEMM (gemm.cu)
 struct GemmPlan {

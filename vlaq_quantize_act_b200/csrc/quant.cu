@@ -490,6 +490,35 @@ cudaError_t launch_quant_fp8(const void* X, int64_t rows, int64_t K, const void*
   return launch_rows<kFp8, kPerRow>(X, rows, K, gamma, eps, flags, codes, K, nullptr, s_out, nullptr, s);
 }
 
+namespace {
+// Tiled (128x4, the layout the tensor cores read) -> row-major [rows, K/16]
+// block scales: one thread per output word of four scale bytes (K/16 may
+// not be a multiple of 4: the last word of a row is written byte-wise).
+__global__ void scales_to_rowmajor_kernel(const uint8_t* __restrict__ in, uint8_t* __restrict__ out, int64_t rows,
+                                          int cols, int nblk64) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int words = (cols + 3) >> 2;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= rows * words) return;
+  const int64_t r = i / words;
+  const int j = static_cast<int>(i % words);  // 64-block j: scale columns 4j .. 4j + 3
+  const uint32_t w = *reinterpret_cast<const uint32_t*>(in + ((r >> 7) * nblk64 + j) * 512 + (r & 31) * 16 +
+                                                        ((r & 127) >> 5) * 4);
+  uint8_t* dst = out + r * cols + 4 * j;
+  for (int b = 0; b < 4 && 4 * j + b < cols; ++b) dst[b] = static_cast<uint8_t>(w >> (8 * b));
+}
+}  // namespace
+
+cudaError_t launch_scales_to_rowmajor(const uint8_t* in, uint8_t* out, int64_t rows, int64_t K, cudaStream_t s) {
+  const int cols = static_cast<int>(K / 16);
+  const int nblk64 = static_cast<int>((K + 63) / 64);
+  const int64_t total = rows * ((cols + 3) / 4);
+  const int threads = 256;
+  return launch_pdl(scales_to_rowmajor_kernel, dim3(static_cast<unsigned int>((total + threads - 1) / threads)),
+                    dim3(threads), 0, s, in, out, rows, cols, nblk64);
+}
+
 cudaError_t read_and_clear_quant_status(unsigned int* out, cudaStream_t s) {
   cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_vlaq_quant_status, sizeof(unsigned int), 0,
                                             cudaMemcpyDeviceToHost, s);
