@@ -622,6 +622,29 @@ def main():
         out["e2e"] = {"value": world * step.flops / (ems / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ems,
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    if not args.quick:
+        # ---------------- offline weight quantization (a1), gate_up weights:
+        # HBM-bound; algorithmic bytes = one bf16 read + codes, scales, g
+        K, N, _, W = data["gate_up"]
+        Wd = W.to(device)
+        wq, ws, wg = vq.alloc_nvfp4(N, K, device, per_tensor=True)
+
+        class _WQ:
+            def run(self, c=0):
+                vq.vlaq_quantize_weight_nvfp4(Wd, N, K, 0, wq, ws, wg)
+
+        wgraph = capture(_WQ())
+        for _ in range(args.warmup):
+            wgraph.replay()
+        torch.cuda.synchronize()
+        wms = time_graph(wgraph, args.steps, dist_on, device)
+        wbytes = 2 * N * K + wq.numel() + ws.numel() + 4
+        out["weight_quant"] = {"unit": "GB/s", "value": wbytes / (wms / 1e3) / 1e9, "ms": wms,
+                               "bytes": wbytes, "frac": wbytes / (wms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                               "peak": peaks["hbm_gbs"],
+                               "shape": f"gate_up W {N}x{K} bf16 -> NVFP4 (amax pass + quantize pass)"}
+        del wgraph, Wd, wq, ws, wg
+
     if args.stack:
         # ---------------- 28-layer stack: one graph of 196 prologue + GEMM pairs
         out["stack"] = {}

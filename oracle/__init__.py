@@ -21,6 +21,8 @@ import numpy as np
 
 F_RMSNORM = 1
 F_HADAMARD64 = 2
+F_SMOOTH_AFTER = 4   # smoothing after the rotation (default: before)
+F_SMOOTH_MUL = 8     # multiply by the smoothing vector (default: divide)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
@@ -51,6 +53,10 @@ def _load():
     lib.vo_wht64_inplace.argtypes = [P, i64]
     lib.vo_transform_row.restype = None
     lib.vo_transform_row.argtypes = [P, i64, P, ctypes.c_float, ctypes.c_uint, P]
+    lib.vo_transform_row_smooth.restype = None
+    lib.vo_transform_row_smooth.argtypes = [P, i64, P, ctypes.c_float, ctypes.c_uint, P, P]
+    lib.vo_quantize_nvfp4_smooth.restype = ctypes.c_int
+    lib.vo_quantize_nvfp4_smooth.argtypes = [P, i64, i64, P, ctypes.c_float, ctypes.c_uint, P, P, P, P]
     lib.vo_quantize_nvfp4.restype = ctypes.c_int
     lib.vo_quantize_nvfp4.argtypes = [P, i64, i64, P, ctypes.c_float, ctypes.c_uint,
                                       ctypes.c_int, P, P, P]
@@ -125,6 +131,16 @@ def transform_row(x_bf16, gamma_bf16=None, eps=1e-6, flags=0) -> np.ndarray:
     return y
 
 
+def transform_row_smooth(x_bf16, smooth_f32, gamma_bf16=None, eps=1e-6, flags=0) -> np.ndarray:
+    """transform_row with per-input-channel smoothing (fp32 [K])."""
+    x = _c(x_bf16, np.uint16)
+    a = _c(smooth_f32, np.float32)
+    g = None if gamma_bf16 is None else _c(gamma_bf16, np.uint16)
+    y = np.empty(x.size, dtype=np.float32)
+    _load().vo_transform_row_smooth(_ptr(x), x.size, _ptr(g), ctypes.c_float(eps), flags, _ptr(a), _ptr(y))
+    return y
+
+
 # ------------------------------------------------------------------- NVFP4
 def quantize_nvfp4(X_bf16, gamma_bf16=None, eps=1e-6, flags=0, per_tensor=False):
     """Returns (codes u8 [rows, K/2], scales u8 [rows, K/16], g f32 [rows] or [1])."""
@@ -138,6 +154,24 @@ def quantize_nvfp4(X_bf16, gamma_bf16=None, eps=1e-6, flags=0, per_tensor=False)
                                    1 if per_tensor else 0, _ptr(codes), _ptr(scales), _ptr(g))
     if rc != 0:
         raise ValueError(f"oracle refused NVFP4 quantization of K={K} flags={flags}")
+    return codes, scales, g
+
+
+def quantize_nvfp4_smooth(X_bf16, smooth_f32, gamma_bf16=None, eps=1e-6, flags=0):
+    """Per-token NVFP4 of activations smoothed per input channel: (codes,
+    scales, g) as quantize_nvfp4."""
+    X = _c(X_bf16, np.uint16)
+    rows, K = X.shape
+    a = _c(smooth_f32, np.float32)
+    assert a.size == K
+    g_in = None if gamma_bf16 is None else _c(gamma_bf16, np.uint16)
+    codes = np.zeros((rows, K // 2), dtype=np.uint8)
+    scales = np.zeros((rows, max(K // 16, 1)), dtype=np.uint8)
+    g = np.zeros(rows, dtype=np.float32)
+    rc = _load().vo_quantize_nvfp4_smooth(_ptr(X), rows, K, _ptr(g_in), ctypes.c_float(eps), flags, _ptr(a),
+                                          _ptr(codes), _ptr(scales), _ptr(g))
+    if rc != 0:
+        raise ValueError(f"oracle refused smoothed NVFP4 quantization of K={K} flags={flags}")
     return codes, scales, g
 
 

@@ -49,6 +49,8 @@
 
 #define VO_F_RMSNORM 1u
 #define VO_F_HADAMARD64 2u
+#define VO_F_SMOOTH_AFTER 4u  /* smoothing after the rotation (default before) */
+#define VO_F_SMOOTH_MUL 8u    /* multiply by the smoothing vector (default divide) */
 
 /* ---------------------------------------------------------------- bf16 -- */
 
@@ -187,8 +189,23 @@ void vo_wht64_inplace(float* y, int64_t K) {
 }
 
 /* bf16 row -> fp32, optional RMSNorm (gain gamma, bf16), optional WHT-64. */
-void vo_transform_row(const uint16_t* x, int64_t K, const uint16_t* gamma,
-                      float eps, unsigned flags, float* y) {
+/*
+ * Per-input-channel smoothing (one fp32 factor a_k per channel), applied to
+ * the normalised row: y_k / a_k (FoldQuant's activation scale divide:
+ * "FoldQuant W8A8/W4A4 inference ...", dequant commit, x' = R(x / a) when
+ * folded before the rotation R, R(x) / a when folded after; OpenVINO commit:
+ * RMSNorm with the folded gain, then the divide, then the rotation) or
+ * y_k * a_k (AWQ's pre_quant_scale, which the activations are multiplied by:
+ * "NVIDIA/TensorRT-Edge-LLM PR #193", the pre_quant_scale commit, and
+ * "Alpamayo 2 Super NVFP4 ...", the AWQ paragraph).  One fp32 operation per
+ * element, correctly rounded.
+ */
+static void smooth_row(float* y, int64_t K, const float* a, unsigned flags) {
+  for (int64_t k = 0; k < K; ++k) y[k] = (flags & VO_F_SMOOTH_MUL) ? y[k] * a[k] : y[k] / a[k];
+}
+
+static void transform_row(const uint16_t* x, int64_t K, const uint16_t* gamma, float eps, unsigned flags,
+                          const float* smooth, float* y) {
   for (int64_t k = 0; k < K; ++k) y[k] = vo_bf16_to_f32(x[k]);
   if (flags & VO_F_RMSNORM) {
     float* g = (float*)malloc(sizeof(float) * (size_t)K);
@@ -199,7 +216,20 @@ void vo_transform_row(const uint16_t* x, int64_t K, const uint16_t* gamma,
     free(t);
     free(g);
   }
+  if (smooth && !(flags & VO_F_SMOOTH_AFTER)) smooth_row(y, K, smooth, flags);
   if (flags & VO_F_HADAMARD64) vo_wht64_inplace(y, K);
+  if (smooth && (flags & VO_F_SMOOTH_AFTER)) smooth_row(y, K, smooth, flags);
+}
+
+void vo_transform_row(const uint16_t* x, int64_t K, const uint16_t* gamma,
+                      float eps, unsigned flags, float* y) {
+  transform_row(x, K, gamma, eps, flags, NULL, y);
+}
+
+/* The row transform with a smoothing vector (NULL: none). */
+void vo_transform_row_smooth(const uint16_t* x, int64_t K, const uint16_t* gamma, float eps, unsigned flags,
+                             const float* smooth, float* y) {
+  transform_row(x, K, gamma, eps, flags, smooth, y);
 }
 
 /* --------------------------------------------------------------- NVFP4 -- */
@@ -243,16 +273,34 @@ static void quant_block16(const float* y, int n, float g, uint8_t* sb8_out,
  * Returns 0, or -1 when K is not a multiple of 16 (64 with the Hadamard
  * flag) or a gamma is missing for RMSNorm.
  */
+static int quantize_nvfp4(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* gamma, float eps,
+                          unsigned flags, const float* smooth, int per_tensor, uint8_t* codes, uint8_t* scales,
+                          float* g);
+
 int vo_quantize_nvfp4(const uint16_t* X, int64_t rows, int64_t K,
                       const uint16_t* gamma, float eps, unsigned flags,
                       int per_tensor, uint8_t* codes, uint8_t* scales,
                       float* g) {
+  return quantize_nvfp4(X, rows, K, gamma, eps, flags, NULL, per_tensor, codes, scales, g);
+}
+
+/* Per-token NVFP4 quantization of activations smoothed per input channel
+ * (smooth: fp32 [K], non-NULL). */
+int vo_quantize_nvfp4_smooth(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* gamma, float eps,
+                             unsigned flags, const float* smooth, uint8_t* codes, uint8_t* scales, float* g) {
+  if (smooth == NULL) return -1;
+  return quantize_nvfp4(X, rows, K, gamma, eps, flags, smooth, 0, codes, scales, g);
+}
+
+static int quantize_nvfp4(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* gamma, float eps,
+                          unsigned flags, const float* smooth, int per_tensor, uint8_t* codes, uint8_t* scales,
+                          float* g) {
   if (K <= 0 || K % 16 != 0) return -1;
   if ((flags & VO_F_HADAMARD64) && K % 64 != 0) return -1;
   if ((flags & VO_F_RMSNORM) && gamma == NULL) return -1;
   float* Y = (float*)malloc(sizeof(float) * (size_t)(rows * K));
   for (int64_t r = 0; r < rows; ++r)
-    vo_transform_row(X + r * K, K, gamma, eps, flags, Y + r * K);
+    transform_row(X + r * K, K, gamma, eps, flags, smooth, Y + r * K);
   float gt = 0.0f;
   if (per_tensor) {
     float A = 0.0f;

@@ -16,6 +16,11 @@ import pytest
 import torch
 
 import oracle
+import synthetic_inputs as si
+
+def bits(t):
+    return si.to_bits(t)
+
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
@@ -393,3 +398,66 @@ def test_decode_identity_dense_product():
     wf = torch.from_numpy(W.view(np.int16)).view(torch.bfloat16).double().numpy()
     ref = xf @ wf.T
     assert np.linalg.norm(Y - ref) / np.linalg.norm(ref) < 0.2
+
+
+# ---------------------------------------------------------------- smoothing
+# Per-input-channel smoothing ("FoldQuant W8A8/W4A4 inference ...", dequant
+# commit: x' = R(x / a) folded before the rotation, R(x) / a after; the AWQ
+# pre_quant_scale multiplies instead: "NVIDIA/TensorRT-Edge-LLM PR #193").
+# Pinned against numpy's IEEE fp32 divide / multiply applied to the
+# separately pinned transform steps.
+
+def _smooth_case(K=192, seed=9):
+    rng = np.random.default_rng(seed)
+    x = torch.from_numpy(rng.standard_normal(K).astype(np.float32) * 3).to(torch.bfloat16)
+    gam = torch.from_numpy((0.5 + rng.random(K)).astype(np.float32)).to(torch.bfloat16)
+    a = np.exp(rng.normal(0, 1, K)).astype(np.float32)   # spread like AWQ scales
+    return si.to_bits(x), si.to_bits(gam), a
+
+
+@pytest.mark.parametrize("mul", [False, True])
+def test_smoothing_before_rotation_is_fp32_elementwise_then_wht(mul):
+    xb, gb, a = _smooth_case()
+    fl = oracle.F_RMSNORM | oracle.F_HADAMARD64 | (oracle.F_SMOOTH_MUL if mul else 0)
+    normed = oracle.transform_row(xb, gb, 1e-6, oracle.F_RMSNORM)
+    z = (normed * a if mul else normed / a).astype(np.float32)
+    want = oracle.wht64(z)
+    got = oracle.transform_row_smooth(xb, a, gb, 1e-6, fl)
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("mul", [False, True])
+def test_smoothing_after_rotation_is_wht_then_fp32_elementwise(mul):
+    xb, gb, a = _smooth_case()
+    fl = oracle.F_RMSNORM | oracle.F_HADAMARD64 | oracle.F_SMOOTH_AFTER | (oracle.F_SMOOTH_MUL if mul else 0)
+    rot = oracle.transform_row(xb, gb, 1e-6, oracle.F_RMSNORM | oracle.F_HADAMARD64)
+    want = (rot * a if mul else rot / a).astype(np.float32)
+    got = oracle.transform_row_smooth(xb, a, gb, 1e-6, fl)
+    assert np.array_equal(got, want)
+
+
+def test_smoothing_without_norm_or_rotation_is_one_fp32_divide():
+    xb, _, a = _smooth_case(K=64)
+    want = (xb.astype(np.uint32) << 16).view(np.float32) / a
+    assert np.array_equal(oracle.transform_row_smooth(xb, a), want.astype(np.float32))
+
+
+@pytest.mark.parametrize("flags", [0, 2, 2 | 4, 8, 2 | 8])
+def test_uniform_power_of_two_smoothing_only_rescales_g(flags):
+    """a = 4 everywhere: the transform scales exactly, so codes and block
+    scales are unchanged and g is scaled by exactly 1/4 (x4 for multiply);
+    before and after the rotation agree."""
+    X = si.projection_activations(256, 6, 3)
+    a = np.full(256, 4.0, np.float32)
+    c0, s0, g0 = oracle.quantize_nvfp4(bits(X), flags=flags & 2)
+    c1, s1, g1 = oracle.quantize_nvfp4_smooth(bits(X), a, flags=flags)
+    assert np.array_equal(c0, c1) and np.array_equal(s0, s1)
+    assert np.array_equal(g1, g0 * (4.0 if flags & 8 else 0.25))
+
+
+def test_unit_smoothing_is_identity():
+    X = si.projection_activations(320, 5, 4)
+    for fl in (0, 4, 8, 12):
+        got = oracle.quantize_nvfp4_smooth(bits(X), np.ones(320, np.float32), flags=fl)
+        want = oracle.quantize_nvfp4(bits(X))
+        assert all(np.array_equal(u, v) for u, v in zip(got, want))
