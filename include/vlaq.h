@@ -93,7 +93,9 @@ typedef enum {
 
 enum {
   VLAQ_F_RMSNORM = 1u << 0,
-  VLAQ_F_HADAMARD64 = 1u << 1
+  VLAQ_F_HADAMARD64 = 1u << 1,
+  VLAQ_F_SMOOTH_AFTER = 1u << 2, /* smoothing after the rotation (default: before) */
+  VLAQ_F_SMOOTH_MUL = 1u << 3    /* multiply by the smoothing factors (default: divide) */
 };
 
 /* Human-readable text of the last error on the calling thread ("" if
@@ -148,6 +150,23 @@ VLAQ_API vlaq_status vlaq_quantize_act_nvfp4(const void* X, int64_t M, int64_t K
                                     uint32_t flags, uint8_t* codes,
                                     uint8_t* scales, float* g_x,
                                     void* stream);
+
+/* vlaq_quantize_act_nvfp4 with per-input-channel smoothing: after the
+ * optional RMSNorm, every channel k is divided by smooth[k] (FoldQuant's
+ * activation scale: "FoldQuant W8A8/W4A4 inference", dequant commit,
+ * x' = R(x / a), or R(x) / a with VLAQ_F_SMOOTH_AFTER, R the block
+ * rotation), or multiplied by it with VLAQ_F_SMOOTH_MUL (AWQ's
+ * pre_quant_scale, which activations are multiplied by: "NVIDIA/TensorRT-
+ * Edge-LLM PR #193", pre_quant_scale commit).  One correctly rounded fp32
+ * operation per element; the weights must carry the inverse factor.
+ *   smooth  fp32 [K] (device, 16-byte aligned), finite and non-zero
+ *   flags   any of VLAQ_F_RMSNORM | VLAQ_F_HADAMARD64 | VLAQ_F_SMOOTH_AFTER
+ *           | VLAQ_F_SMOOTH_MUL
+ * Other arguments, outputs and limits as vlaq_quantize_act_nvfp4. */
+VLAQ_API vlaq_status vlaq_quantize_act_nvfp4_smooth(const void* X, int64_t M, int64_t K,
+                                            const void* gamma, const float* smooth,
+                                            float eps, uint32_t flags, uint8_t* codes,
+                                            uint8_t* scales, float* g_x, void* stream);
 
 /* Block scales from the 128x4 tiled layout the GEMM reads (as written by
  * the NVFP4 quantizers, vlaq_nvfp4_scale_bytes(rows, K) bytes) to the

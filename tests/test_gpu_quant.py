@@ -171,3 +171,32 @@ def test_scales_to_rowmajor_random_buffer():
     m.vlaq_scales_to_rowmajor(to_dev(buf), out, rows, K)
     torch.cuda.synchronize()
     assert np.array_equal(out.cpu().numpy(), layouts.untile_scales(buf, rows, K))
+
+
+def _awq_like_smoothing(K, seed):
+    """Per-channel factors spread like the AWQ scales the pages report for
+    Qwen2.5-VL-7B (0.1553 .. 6.4375, log-uniform here)."""
+    rng = np.random.default_rng(seed)
+    return np.exp(rng.uniform(np.log(0.1553), np.log(6.4375), K)).astype(np.float32)
+
+
+# (M, K, transform flags): ragged K (no rotation), several 64-blocks, the
+# 16-warp row kernel, and full-size rows of the qkv and down inputs
+SMOOTH_CASES = [(5, 336, 0), (37, 1024, 0), (37, 1024, 3), (9, 18944, 2), (1024, 3584, 3), (256, 18944, 0)]
+
+
+@pytest.mark.parametrize("M,K,tf", SMOOTH_CASES)
+@pytest.mark.parametrize("mode", [0, 4, 8, 12])
+def test_act_nvfp4_smooth_vs_oracle(M, K, tf, mode):
+    m = vq()
+    X = si.projection_activations(K, M, 71)
+    gam = si.norm_gain(K, 71)
+    a = _awq_like_smoothing(K, 72)
+    flags = tf | mode
+    xq, xs, xg = m.alloc_nvfp4(M, K)
+    m.vlaq_quantize_act_nvfp4_smooth(X.cuda(), M, K, gam.cuda(), to_dev(a), 1e-6, flags, xq, xs, xg)
+    torch.cuda.synchronize()
+    m.vlaq_check()
+    ref = oracle.quantize_nvfp4_smooth(bits(X), a, bits(gam), 1e-6, flags)
+    assert_nvfp4_equal((xq.cpu().numpy(), xs.cpu().numpy(), xg.cpu().numpy()), ref, M, K,
+                       f"smooth M={M} K={K} flags={flags}")

@@ -17,7 +17,7 @@ import os
 import torch
 
 __all__ = [
-    "VlaqError", "F_RMSNORM", "F_HADAMARD64", "LIB_PATH",
+    "VlaqError", "F_RMSNORM", "F_HADAMARD64", "F_SMOOTH_AFTER", "F_SMOOTH_MUL", "LIB_PATH",
     "vlaq_last_error", "vlaq_version", "vlaq_check",
     "vlaq_nvfp4_code_pitch", "vlaq_nvfp4_scale_bytes", "vlaq_linear_workspace_bytes",
     "vlaq_quantize_weight_nvfp4", "vlaq_quantize_act_nvfp4", "vlaq_linear_nvfp4",
@@ -27,6 +27,8 @@ __all__ = [
 
 F_RMSNORM = 1
 F_HADAMARD64 = 2
+F_SMOOTH_AFTER = 4
+F_SMOOTH_MUL = 8
 
 STATUS_NAMES = {
     0: "VLAQ_OK", 1: "VLAQ_ERR_INVALID_ARG", 2: "VLAQ_ERR_SHAPE", 3: "VLAQ_ERR_ALIGN",
@@ -61,6 +63,7 @@ _SIGS = {
     "vlaq_linear_fp8": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "vlaq_linear_nvfp4_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "vlaq_scales_to_rowmajor": (ctypes.c_int, [_P, _P, _I64, _I64, _P]),
+    "vlaq_quantize_act_nvfp4_smooth": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _F, _U32, _P, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -130,6 +133,11 @@ def vlaq_quantize_weight_nvfp4(W, N, K, flags, codes, scales, g_w, stream=None):
 def vlaq_quantize_act_nvfp4(X, M, K, gamma, eps, flags, codes, scales, g_x, stream=None):
     _check(_lib.vlaq_quantize_act_nvfp4(_ptr(X), M, K, _ptr(gamma), eps, flags, _ptr(codes), _ptr(scales),
                                         _ptr(g_x), _stream(stream)))
+
+
+def vlaq_quantize_act_nvfp4_smooth(X, M, K, gamma, smooth, eps, flags, codes, scales, g_x, stream=None):
+    _check(_lib.vlaq_quantize_act_nvfp4_smooth(_ptr(X), M, K, _ptr(gamma), _ptr(smooth), eps, flags, _ptr(codes),
+                                               _ptr(scales), _ptr(g_x), _stream(stream)))
 
 
 def vlaq_scales_to_rowmajor(scales, out, rows, K, stream=None):

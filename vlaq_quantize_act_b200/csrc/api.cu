@@ -152,6 +152,30 @@ vlaq_status vlaq_quantize_act_nvfp4(const void* X, int64_t M, int64_t K, const v
   return ok();
 }
 
+vlaq_status vlaq_quantize_act_nvfp4_smooth(const void* X, int64_t M, int64_t K, const void* gamma,
+                                           const float* smooth, float eps, uint32_t flags, uint8_t* codes,
+                                           uint8_t* scales, float* g_x, void* stream) {
+  const char* fn = "vlaq_quantize_act_nvfp4_smooth";
+  vlaq_status st;
+  if ((st = check_flags(fn, flags, VLAQ_F_RMSNORM | VLAQ_F_HADAMARD64 | VLAQ_F_SMOOTH_AFTER | VLAQ_F_SMOOTH_MUL)))
+    return st;
+  if ((st = check_k(fn, K, flags, true, vlaq::kMaxQuantK))) return st;
+  if (M < 0) return fail(VLAQ_ERR_INVALID_ARG, "%s: M = %lld is negative", fn, (long long)M);
+  if (M > 0x7FFFFFFF) return fail(VLAQ_ERR_SHAPE, "%s: M = %lld is too large", fn, (long long)M);
+  if (M == 0) return ok();
+  VLAQ_NONNULL(fn, X);
+  VLAQ_NONNULL(fn, smooth);
+  VLAQ_NONNULL(fn, codes);
+  VLAQ_NONNULL(fn, scales);
+  VLAQ_NONNULL(fn, g_x);
+  if (flags & VLAQ_F_RMSNORM) VLAQ_NONNULL(fn, gamma);
+  if ((st = check_device(fn))) return st;
+  cudaError_t e = vlaq::launch_quant_act_nvfp4_smooth(X, M, K, gamma, smooth, eps, flags, codes, scales, g_x,
+                                                      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(fn, e);
+  return ok();
+}
+
 vlaq_status vlaq_quantize_weight_nvfp4(const void* W, int64_t N, int64_t K, uint32_t flags, uint8_t* codes,
                                        uint8_t* scales, float* g_w, void* stream) {
   const char* fn = "vlaq_quantize_weight_nvfp4";

@@ -21,6 +21,8 @@ constexpr long long kWaitBudgetCycles = 2000000000LL;
 
 constexpr uint32_t kFlagRmsNorm = 1u;
 constexpr uint32_t kFlagHadamard = 2u;
+constexpr uint32_t kFlagSmoothAfter = 4u;  // smoothing after the rotation (default: before)
+constexpr uint32_t kFlagSmoothMul = 8u;    // multiply by the smoothing factors (default: divide)
 
 inline int64_t nvfp4_code_pitch(int64_t K) { return (K + 63) / 64 * 32; }
 inline int64_t nvfp4_scale_cols_padded(int64_t K) { return (K + 63) / 64 * 4; }
@@ -30,6 +32,9 @@ inline int64_t nvfp4_rows_padded(int64_t rows) { return (rows + 127) / 128 * 128
 cudaError_t launch_quant_act_nvfp4(const void* X, int64_t M, int64_t K, const void* gamma, float eps,
                                    uint32_t flags, uint8_t* codes, uint8_t* scales, float* g_x,
                                    cudaStream_t s);
+cudaError_t launch_quant_act_nvfp4_smooth(const void* X, int64_t M, int64_t K, const void* gamma,
+                                          const float* smooth, float eps, uint32_t flags, uint8_t* codes,
+                                          uint8_t* scales, float* g_x, cudaStream_t s);
 cudaError_t launch_quant_weight_nvfp4(const void* W, int64_t N, int64_t K, uint32_t flags,
                                       uint8_t* codes, uint8_t* scales, float* g_w, cudaStream_t s);
 cudaError_t launch_quant_fp8(const void* X, int64_t rows, int64_t K, const void* gamma, float eps,

@@ -145,6 +145,8 @@ struct RowArgs {
   float* gout;
   unsigned int* amax_word;
   int64_t rows;
+  const float* smooth;  // per-input-channel smoothing factors [K] (or null)
+  uint32_t sflags;      // kFlagSmoothAfter | kFlagSmoothMul
   int nbuf;       // ring depth (rows in flight per CTA)
   int row_bytes;  // ring slot size (2 K rounded up to 128)
   long long budget;
@@ -179,9 +181,23 @@ __device__ __forceinline__ void wht64_lanes(float* v, int lane) {
   for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], 0.125f);
 }
 
+// y_k / a_k or y_k * a_k for the 16 channels of block q (smoothing).
+__device__ __forceinline__ void smooth_block(const RowArgs& a, int q, float* v) {
+  const float4* s4 = reinterpret_cast<const float4*>(a.smooth) + 4 * q;
+  const bool mul = (a.sflags & kFlagSmoothMul) != 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 f = __ldg(s4 + i);
+    const float fs[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[4 * i + j] = mul ? __fmul_rn(v[4 * i + j], fs[j]) : __fdiv_rn(v[4 * i + j], fs[j]);
+  }
+}
+
 // The 16 values of block q after the row transform (zeros past the row):
-// y = (x r) gamma for RMSNorm, then the block-64 WHT.  Warp-uniform.
-template <bool NORM, bool WHT>
+// y = (x r) gamma for RMSNorm, the smoothing divide (or multiply) before or
+// after the block-64 WHT.  Warp-uniform.
+template <bool NORM, bool WHT, bool SMOOTH>
 __device__ __forceinline__ void block_values(const RowArgs& a, const uint8_t* rs, int q, int nblk16, float r,
                                              int lane, float* v) {
   if (q < nblk16) {
@@ -196,11 +212,13 @@ __device__ __forceinline__ void block_values(const RowArgs& a, const uint8_t* rs
 #pragma unroll
       for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(__fmul_rn(v[j], r), gm[j]);
     }
+    if (SMOOTH && !(a.sflags & kFlagSmoothAfter)) smooth_block(a, q, v);
   } else {
 #pragma unroll
     for (int j = 0; j < 16; ++j) v[j] = 0.0f;
   }
   if (WHT) wht64_lanes(v, lane);
+  if (SMOOTH && (a.sflags & kFlagSmoothAfter) && q < nblk16) smooth_block(a, q, v);
 }
 
 __device__ __forceinline__ float absmax16(const float* v) {
@@ -214,7 +232,7 @@ __device__ __forceinline__ float absmax16(const float* v) {
 // amax pass, tensor quantize pass), NORM (RMSNorm, per-row modes only), WHT
 // (block-64 Hadamard), W warps per CTA.  Persistent grid: the CTA takes rows
 // blockIdx.x + i gridDim.x, the ring slot of row i is i mod nbuf.
-template <int FMT, int MODE, bool NORM, bool WHT, int W>
+template <int FMT, int MODE, bool NORM, bool WHT, bool SMOOTH, int W>
 __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) quant_rows_kernel(const RowArgs a) {
   constexpr int T = RowCfg<W>::kThreads;
   constexpr int MAXIT = (W == 8 ? kShortRowK : int(kMaxQuantK)) / 16 / T;  // blocks per lane, at most
@@ -309,9 +327,9 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
         if (it < iters) {
           const int q = (it * W + warp) * 32 + lane;
           float m = 0.0f;
-          if (NORM || WHT) {
+          if (NORM || WHT || SMOOTH) {
             float v[16];
-            block_values<NORM, WHT>(a, rs, q, nblk16, r, lane, v);
+            block_values<NORM, WHT, SMOOTH>(a, rs, q, nblk16, r, lane, v);
             m = absmax16(v);
           } else if (q < nblk16) {
             const uint4* src = reinterpret_cast<const uint4*>(rs) + 2 * q;
@@ -347,7 +365,7 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
           if (it < iters) {
             const int q = (it * W + warp) * 32 + lane;
             float v[16];
-            block_values<NORM, WHT>(a, rs, q, nblk16, r, lane, v);
+            block_values<NORM, WHT, SMOOTH>(a, rs, q, nblk16, r, lane, v);
             const float a16 = (MODE == kPerRow) ? a16r[it] : absmax16(v);
             uint32_t sb8 = 0;
             float S = 0.0f;
@@ -373,7 +391,7 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
           if (it < iters) {
             const int q = (it * W + warp) * 32 + lane;
             float v[16];
-            block_values<NORM, WHT>(a, rs, q, nblk16, r, lane, v);
+            block_values<NORM, WHT, SMOOTH>(a, rs, q, nblk16, r, lane, v);
             float qv[16];
             quotients<16>(v, dg, qv);
             uint32_t w[4];
@@ -409,10 +427,10 @@ __global__ void finalize_global_kernel(float* g) {
   g[0] = __fdiv_rn(__uint_as_float(*reinterpret_cast<unsigned int*>(g)), 2688.0f);
 }
 
-template <int FMT, int MODE, bool NORM, bool WHT, int W>
+template <int FMT, int MODE, bool NORM, bool WHT, bool SMOOTH, int W>
 cudaError_t launch_ring(RowArgs a, cudaStream_t s) {
   using C = RowCfg<W>;
-  auto kern = quant_rows_kernel<FMT, MODE, NORM, WHT, W>;
+  auto kern = quant_rows_kernel<FMT, MODE, NORM, WHT, SMOOTH, W>;
   const int fit = C::kRingBytes / a.row_bytes;
   a.nbuf = fit < 2 ? 2 : (fit > kMaxRowBufs ? kMaxRowBufs : fit);  // 2 x 64 KiB at the largest K
   const size_t smem = static_cast<size_t>(a.nbuf) * a.row_bytes;
@@ -429,16 +447,16 @@ cudaError_t launch_ring(RowArgs a, cudaStream_t s) {
   return launch_pdl(kern, dim3(grid), dim3(C::kThreads), smem, s, a);
 }
 
-template <int FMT, int MODE, bool NORM, bool WHT>
+template <int FMT, int MODE, bool NORM, bool WHT, bool SMOOTH = false>
 cudaError_t launch_shape(const RowArgs& a, cudaStream_t s) {
-  if (a.K <= kShortRowK) return launch_ring<FMT, MODE, NORM, WHT, 8>(a, s);
-  return launch_ring<FMT, MODE, NORM, WHT, 16>(a, s);
+  if (a.K <= kShortRowK) return launch_ring<FMT, MODE, NORM, WHT, SMOOTH, 8>(a, s);
+  return launch_ring<FMT, MODE, NORM, WHT, SMOOTH, 16>(a, s);
 }
 
 template <int FMT, int MODE>
 cudaError_t launch_rows(const void* X, int64_t rows, int64_t K, const void* gamma, float eps, uint32_t flags,
                         uint8_t* codes, int64_t pitch, uint8_t* scales, float* gout, unsigned int* amax,
-                        cudaStream_t s) {
+                        cudaStream_t s, const float* smooth = nullptr) {
   RowArgs a;
   a.X = static_cast<const __nv_bfloat16*>(X);
   a.K = static_cast<int>(K);
@@ -450,10 +468,19 @@ cudaError_t launch_rows(const void* X, int64_t rows, int64_t K, const void* gamm
   a.gout = gout;
   a.amax_word = amax;
   a.rows = rows;
+  a.smooth = smooth;
+  a.sflags = flags & (kFlagSmoothAfter | kFlagSmoothMul);
   a.nbuf = 0;
   a.row_bytes = static_cast<int>((2 * K + 127) / 128 * 128);
   a.budget = kWaitBudgetCycles;
   const bool wht = (flags & kFlagHadamard) != 0;
+  if constexpr (MODE == kPerRow && FMT == kNvfp4) {
+    if (smooth) {
+      if (flags & kFlagRmsNorm)
+        return wht ? launch_shape<FMT, MODE, true, true, true>(a, s) : launch_shape<FMT, MODE, true, false, true>(a, s);
+      return wht ? launch_shape<FMT, MODE, false, true, true>(a, s) : launch_shape<FMT, MODE, false, false, true>(a, s);
+    }
+  }
   if constexpr (MODE == kPerRow) {
     if (flags & kFlagRmsNorm)
       return wht ? launch_shape<FMT, MODE, true, true>(a, s) : launch_shape<FMT, MODE, true, false>(a, s);
@@ -467,6 +494,13 @@ cudaError_t launch_quant_act_nvfp4(const void* X, int64_t M, int64_t K, const vo
                                    uint32_t flags, uint8_t* codes, uint8_t* scales, float* g_x, cudaStream_t s) {
   return launch_rows<kNvfp4, kPerRow>(X, M, K, gamma, eps, flags, codes, nvfp4_code_pitch(K), scales, g_x, nullptr,
                                       s);
+}
+
+cudaError_t launch_quant_act_nvfp4_smooth(const void* X, int64_t M, int64_t K, const void* gamma, const float* smooth,
+                                          float eps, uint32_t flags, uint8_t* codes, uint8_t* scales, float* g_x,
+                                          cudaStream_t s) {
+  return launch_rows<kNvfp4, kPerRow>(X, M, K, gamma, eps, flags, codes, nvfp4_code_pitch(K), scales, g_x, nullptr,
+                                      s, smooth);
 }
 
 cudaError_t launch_quant_weight_nvfp4(const void* W, int64_t N, int64_t K, uint32_t flags, uint8_t* codes,
