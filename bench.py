@@ -623,6 +623,40 @@ def main():
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if not args.quick:
+        # ---------------- prologue variants over the four projection inputs:
+        # fused RMSNorm + block-64 rotation, per-channel smoothing (divide,
+        # before the rotation), and both; same bytes as the plain prologue
+        # (the gains and smoothing factors stay in cache)
+        variants = {"fused_rmsnorm_wht": (3, False), "smooth": (0, True), "fused_smooth": (3, True)}
+        extra = {}
+        for L in step.layers:
+            K = L["K"]
+            rng = np.random.default_rng(K)
+            extra[L["name"]] = (si.norm_gain(K, 5).to(device),
+                                torch.from_numpy(np.exp(rng.uniform(np.log(0.1553), np.log(6.4375), K))
+                                                 .astype(np.float32)).to(device))
+        out["prologue_variants"] = {}
+        for vname, (vflags, vsmooth) in variants.items():
+            class _PV:
+                def run(self, c=0):
+                    for L in step.layers:
+                        xq, xs, xg = L["act"]
+                        gam, sm = extra[L["name"]]
+                        if vsmooth:
+                            vq.vlaq_quantize_act_nvfp4_smooth(L["X"], M_PREFILL, L["K"], gam, sm, 1e-6, vflags,
+                                                              xq, xs, xg)
+                        else:
+                            vq.vlaq_quantize_act_nvfp4(L["X"], M_PREFILL, L["K"], gam, 1e-6, vflags, xq, xs, xg)
+
+            pgraph = capture(_PV())
+            for _ in range(args.warmup):
+                pgraph.replay()
+            torch.cuda.synchronize()
+            pms = time_graph(pgraph, args.steps, dist_on, device)
+            out["prologue_variants"][vname] = {"GB/s": pro_bytes / (pms / 1e3) / 1e9, "ms": pms,
+                                               "frac": pro_bytes / (pms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+            del pgraph
+
         # ---------------- offline weight quantization (a1), gate_up weights:
         # HBM-bound; algorithmic bytes = one bf16 read + codes, scales, g
         K, N, _, W = data["gate_up"]
