@@ -67,20 +67,30 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def traffic_source_sha(sources):
+    """sha256 (16 hex digits) of the source the traffic counters depend on:
+    a list of {"file": path, optional "from" / "to" markers bounding a
+    region of the file}."""
+    import hashlib
+    h = hashlib.sha256()
+    for src in sources:
+        txt = open(os.path.join(ROOT, src["file"]), encoding="utf-8").read()
+        if "from" in src:
+            a = txt.index(src["from"])
+            txt = txt[a:txt.index(src["to"], a)]
+        h.update(txt.encode())
+    return h.hexdigest()[:16]
+
+
 def load_traffic(kernel_key):
     """dram bytes per launch from the committed ncu summary, valid only while
-    the kernel source is unchanged (hash recorded beside the counters)."""
+    the kernel's source is unchanged (hash recorded beside the counters)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     try:
-        d = json.load(open(p))
-        ent = d.get(kernel_key)
-        if not ent:
-            return None
-        import hashlib
-        src = open(os.path.join(ROOT, ent["source"]), "rb").read()
-        if hashlib.sha256(src).hexdigest()[:16] != ent["source_sha"]:
+        ent = json.load(open(p)).get(kernel_key)
+        if not ent or traffic_source_sha(ent["sources"]) != ent["source_sha"]:
             return None
         return ent["bytes_per_launch"]
     except Exception:

@@ -112,6 +112,14 @@ VLAQ_API int vlaq_version(void);
  * bounded wait since the last check, VLAQ_ERR_CUDA on a CUDA error. */
 VLAQ_API vlaq_status vlaq_check(void* stream);
 
+/* Failure-path self test: launches one kernel whose bounded wait on an
+ * mbarrier that nothing arrives on runs out after about 1 ms; it records
+ * the timeout in the device status word exactly as the GEMM and quantizer
+ * kernels do, so the next vlaq_check(stream) returns VLAQ_ERR_TIMEOUT and
+ * the one after it VLAQ_OK.  No copy, MMA or tensor memory is involved; the
+ * context stays usable. */
+VLAQ_API vlaq_status vlaq_selftest_wait_timeout(void* stream);
+
 /* ----------------------------------------------------------- size helpers */
 VLAQ_API int64_t vlaq_nvfp4_code_pitch(int64_t K);               /* bytes per row   */
 VLAQ_API int64_t vlaq_nvfp4_scale_bytes(int64_t rows, int64_t K);/* tiled scales    */

@@ -63,6 +63,7 @@ _SIGS = {
     "vlaq_linear_fp8": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "vlaq_linear_nvfp4_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "vlaq_scales_to_rowmajor": (ctypes.c_int, [_P, _P, _I64, _I64, _P]),
+    "vlaq_selftest_wait_timeout": (ctypes.c_int, [_P]),
     "vlaq_quantize_act_nvfp4_smooth": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _F, _U32, _P, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -138,6 +139,10 @@ def vlaq_quantize_act_nvfp4(X, M, K, gamma, eps, flags, codes, scales, g_x, stre
 def vlaq_quantize_act_nvfp4_smooth(X, M, K, gamma, smooth, eps, flags, codes, scales, g_x, stream=None):
     _check(_lib.vlaq_quantize_act_nvfp4_smooth(_ptr(X), M, K, _ptr(gamma), _ptr(smooth), eps, flags, _ptr(codes),
                                                _ptr(scales), _ptr(g_x), _stream(stream)))
+
+
+def vlaq_selftest_wait_timeout(stream=None):
+    _check(_lib.vlaq_selftest_wait_timeout(_stream(stream)))
 
 
 def vlaq_scales_to_rowmajor(scales, out, rows, K, stream=None):

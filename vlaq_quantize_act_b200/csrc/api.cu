@@ -131,6 +131,15 @@ vlaq_status vlaq_check(void* stream) {
   return ok();
 }
 
+vlaq_status vlaq_selftest_wait_timeout(void* stream) {
+  const char* fn = "vlaq_selftest_wait_timeout";
+  vlaq_status st;
+  if ((st = check_device(fn))) return st;
+  cudaError_t e = vlaq::launch_selftest_wait_timeout(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(fn, e);
+  return ok();
+}
+
 vlaq_status vlaq_quantize_act_nvfp4(const void* X, int64_t M, int64_t K, const void* gamma, float eps,
                                     uint32_t flags, uint8_t* codes, uint8_t* scales, float* g_x, void* stream) {
   const char* fn = "vlaq_quantize_act_nvfp4";

@@ -5,21 +5,19 @@
 //             = sum_k e4m3(x[m, k]) e4m3(w[n, k])                                 (FP8)
 //   scale = g_x[m] * g_w (NVFP4) or s_x[m] * s_w[n] (FP8)
 //
-// Persistent, warp-specialised kernel, one CTA per SM:
-//   warp 0      TMA producer: 2-D tiled loads of the packed codes (128-byte
-//               swizzle) and 1-D bulk loads of the 512-byte scale atoms into
-//               a ring of shared-memory stages;
-//   warp 1      allocates TMEM and issues, from one thread, tcgen05.cp of the
-//               scale atoms into TMEM and tcgen05.mma (kind::mxf4nvf4 with
-//               block-16 UE4M3 scale vectors, or kind::f8f6f4) accumulating
-//               a 128 x BN fp32 tile in TMEM; tcgen05.commit frees stages
-//               and hands finished accumulators to the epilogue;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (double-buffered in
-//               TMEM so the next tile's MMAs overlap), scale, residual add,
-//               bf16 round, 16-byte global stores.
-// Split-K (decode shapes, few output tiles): each split writes fp32 partial
-// sums to the caller's workspace and a small kernel reduces them in fixed
-// order and applies the same epilogue.
+// Two persistent, warp-specialised kernels, one CTA per SM, both fed by TMA
+// (2-D tiled loads of the packed codes with 128-byte swizzle) through a ring
+// of shared-memory stages, accumulating 128 x BN fp32 tiles in TMEM with
+// tcgen05.mma issued from one thread:
+//   gemm_fp4_sfw_kernel  NVFP4, 128 x 256 tiles, kind::mxf4nvf4 with block-16
+//                        UE4M3 scale vectors that four warps write into TMEM;
+//                        split-K (decode shapes) reduced in-kernel by the
+//                        last split of each tile;
+//   gemm_fp8_kernel<BN>  FP8 E4M3, kind::f8f6f4, 128 x 256 or 128 x 128 tiles
+//                        (double-buffered accumulator); split-K partials are
+//                        added by splitk_reduce_kernel in fixed order.
+// Epilogues: tcgen05.ld of the accumulator, scale, residual add, bf16 round,
+// global stores.
 //
 // Every mbarrier wait is bounded (clock budget); a wait that runs out sets a
 // shared abort flag and the device status word, the roles drain their own
@@ -42,28 +40,23 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kTmemCols = 512;
 
-template <bool FP4, int BN>
-struct Cfg {
+// FP8 kernel shape: tile 128 x BN, stages of K = 128 E4M3 elements.
+template <int BN>
+struct Fp8Cfg {
   static constexpr int A_BYTES = kBM * 128;
   static constexpr int B_BYTES = BN * 128;
-  static constexpr int NRB = BN / 128;                  // 128-row scale blocks per B tile
-  static constexpr int SFA_BYTES = FP4 ? 4 * 512 : 0;   // 4 k-atoms
-  static constexpr int SFB_BYTES = FP4 ? NRB * 4 * 512 : 0;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int NRB = BN / 128;                  // 128-column halves of the tile
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (220 * 1024) / STAGE_BYTES > 8 ? 8 : (220 * 1024) / STAGE_BYTES;
   static constexpr int ACC_BUFS = (BN <= 128) ? 2 : 1;
-  static constexpr int SFA_COL = ACC_BUFS * BN;         // 2 buffers x 16 columns
-  static constexpr int SFB_COL = SFA_COL + 32;          // 2 buffers x NRB*16 columns
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
   // one epilogue warp per (TMEM sub-partition, 128-column half)
   static constexpr int EPI_WARPS = 4 * NRB;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-  static_assert(SFB_COL + 2 * NRB * 16 <= kTmemCols, "TMEM budget");
+  static_assert(ACC_BUFS * BN <= kTmemCols, "TMEM budget");
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
-  // Instruction descriptors (M = 128, N = BN, K-major A and B).
-  static constexpr uint32_t IDESC =
-      FP4 ? ((1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBM >> 4) << 24))
-          : ((1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBM >> 4) << 24));
+  // instruction descriptor: kind::f8f6f4, E4M3 x E4M3, fp32 D, M = 128, N = BN
+  static constexpr uint32_t IDESC = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
 };
 
 struct GemmArgs {
@@ -199,11 +192,14 @@ __device__ __forceinline__ void store_output(const GemmArgs& a, int row, int col
   }
 }
 
-template <bool FP4, int BN>
-__global__ void __launch_bounds__(Cfg<FP4, BN>::THREADS, 1)
-gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-            const GemmArgs args) {
-  using C = Cfg<FP4, BN>;
+// FP8 E4M3 W8A8 GEMM: 64 + 32 EPI_WARPS threads, warp 0 TMA producer, warp
+// 1 TMEM allocator and MMA issuer (kind::f8f6f4), the rest epilogue warps;
+// split-K partials are added by splitk_reduce_kernel.
+template <int BN>
+__global__ void __launch_bounds__(Fp8Cfg<BN>::THREADS, 1)
+gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const GemmArgs args) {
+  using C = Fp8Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[C::STAGES];
   __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
@@ -263,28 +259,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           }
           uint8_t* sa = smem + stage * C::STAGE_BYTES;
           uint8_t* sb = sa + C::A_BYTES;
-          const int steps = min(4, args.k_steps - 4 * kt);
-          uint32_t bytes = C::A_BYTES + C::B_BYTES;
-          int nrb = 0;
-          if (FP4) {
-            nrb = min(C::NRB, args.w_row_blocks - w.n * C::NRB);
-            bytes += static_cast<uint32_t>(steps * 512 * (1 + nrb));
-          }
-          mbar_arrive_expect_tx(&full_bar[stage], bytes);
+          mbar_arrive_expect_tx(&full_bar[stage], C::A_BYTES + C::B_BYTES);
           armed |= 1u << stage;
           armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
           tma_load_2d(sa, &tmA, &full_bar[stage], kt * 128, w.m * kBM);
           tma_load_2d(sb, &tmB, &full_bar[stage], kt * 128, w.n * BN);
-          if (FP4) {
-            uint8_t* ssfa = sb + C::B_BYTES;
-            uint8_t* ssfb = ssfa + C::SFA_BYTES;
-            bulk_load(ssfa, args.xs + (static_cast<size_t>(w.m) * args.ka + 4 * kt) * 512,
-                      steps * 512, &full_bar[stage]);
-            for (int rb = 0; rb < nrb; ++rb)
-              bulk_load(ssfb + rb * 2048,
-                        args.ws + (static_cast<size_t>(w.n * C::NRB + rb) * args.ka + 4 * kt) * 512,
-                        steps * 512, &full_bar[stage]);
-          }
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -309,7 +288,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      uint32_t sf_buf = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
         const Unit w = decode_unit(args, u);
@@ -328,32 +306,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           uint8_t* sa = smem + stage * C::STAGE_BYTES;
           uint8_t* sb = sa + C::A_BYTES;
           const int steps = min(4, args.k_steps - 4 * kt);
-          const uint32_t sfa_base = tmem + C::SFA_COL + sf_buf * 16;
-          const uint32_t sfb_base = tmem + C::SFB_COL + sf_buf * (C::NRB * 16);
-          if (FP4) {
-            const uint32_t ssfa = smem_u32(sb + C::B_BYTES);
-            const uint32_t ssfb = ssfa + C::SFA_BYTES;
-            for (int j = 0; j < steps; ++j) {
-              tmem_cp_32x128b_warpx4(sfa_base + 4 * j, sdesc_sf_block(ssfa + 512 * j));
-#pragma unroll
-              for (int rb = 0; rb < C::NRB; ++rb)
-                tmem_cp_32x128b_warpx4(sfb_base + C::NRB * 4 * j + 4 * rb,
-                                       sdesc_sf_block(ssfb + rb * 2048 + 512 * j));
-            }
-          }
           const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
-          for (int j = 0; j < steps; ++j) {
-            const uint64_t ad = sdesc_kmajor_sw128(a0 + 32 * j);
-            const uint64_t bd = sdesc_kmajor_sw128(b0 + 32 * j);
-            const uint32_t accum = (kt > w.kt0 || j > 0) ? 1u : 0u;
-            if (FP4)
-              mma_mxf4nvf4(d_tmem, ad, bd, C::IDESC, sfa_base + 4 * j, sfb_base + C::NRB * 4 * j,
-                           accum);
-            else
-              mma_f8f6f4(d_tmem, ad, bd, C::IDESC, accum);
-          }
+          for (int j = 0; j < steps; ++j)
+            mma_f8f6f4(d_tmem, sdesc_kmajor_sw128(a0 + 32 * j), sdesc_kmajor_sw128(b0 + 32 * j), C::IDESC,
+                       (kt > w.kt0 || j > 0) ? 1u : 0u);
           umma_commit(&empty_bar[stage]);
-          sf_buf ^= 1u;
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -406,7 +363,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         acc_phase ^= 1u;
       }
       float rs = 0.0f;
-      if (row_ok && args.splits == 1) rs = FP4 ? args.xg[row] * args.wg[0] : args.xg[row];
+      if (row_ok && args.splits == 1) rs = args.xg[row];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int col0 = w.n * BN + 128 * h + 32 * c;
@@ -414,7 +371,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           if (args.splits > 1)
             store_partial(args, w.split, row, col0, r[c]);
           else
-            store_output<FP4>(args, row, col0, rs, r[c]);
+            store_output<false>(args, row, col0, rs, r[c]);
         }
       }
     }
@@ -898,16 +855,10 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t r
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool FP4, int BN>
-cudaError_t run(const uint8_t* xq, const uint8_t* xs, const float* xg, const uint8_t* wq, const uint8_t* ws,
-                const float* wg, const void* residual, void* Y, int64_t M, int64_t N, int64_t K,
-                void* workspace, const GemmPlan& plan, long long budget, cudaStream_t s) {
-  using C = Cfg<FP4, BN>;
-  const int64_t pitch = FP4 ? nvfp4_code_pitch(K) : K;
-  CUtensorMap ta, tb;
-  if (!make_map(&ta, xq, static_cast<uint64_t>(pitch), static_cast<uint64_t>(M), static_cast<uint64_t>(pitch), kBM) ||
-      !make_map(&tb, wq, static_cast<uint64_t>(pitch), static_cast<uint64_t>(N), static_cast<uint64_t>(pitch), BN))
-    return cudaErrorInvalidValue;
+// Launch arguments shared by both GEMM kernels (BN: tile width).
+GemmArgs make_args(bool fp4, int BN, const uint8_t* xs, const float* xg, const uint8_t* ws, const float* wg,
+                   const void* residual, void* Y, int64_t M, int64_t N, int64_t K, void* workspace,
+                   const GemmPlan& plan, long long budget) {
   GemmArgs a;
   a.xs = xs;
   a.ws = ws;
@@ -915,13 +866,14 @@ cudaError_t run(const uint8_t* xq, const uint8_t* xs, const float* xg, const uin
   a.wg = wg;
   a.residual = static_cast<const __nv_bfloat16*>(residual);
   a.Y = static_cast<__nv_bfloat16*>(Y);
+  // split-K workspace: tile counters first (NVFP4), then the partial sums
   a.partial = plan.splits > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kSplitCounterBytes)
                               : nullptr;
-  a.counters = nullptr;
+  a.counters = (fp4 && plan.splits > 1) ? static_cast<unsigned int*>(workspace) : nullptr;
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.K = static_cast<int>(K);
-  a.k_steps = static_cast<int>(FP4 ? (K + 63) / 64 : (K + 31) / 32);
+  a.k_steps = static_cast<int>(fp4 ? (K + 63) / 64 : (K + 31) / 32);
   a.k_tiles = (a.k_steps + 3) / 4;
   a.m_tiles = static_cast<int>((M + kBM - 1) / kBM);
   a.n_tiles = static_cast<int>((N + BN - 1) / BN);
@@ -930,26 +882,48 @@ cudaError_t run(const uint8_t* xq, const uint8_t* xs, const float* xg, const uin
   a.ka = static_cast<int>((K + 63) / 64);
   a.w_row_blocks = static_cast<int>((N + 127) / 128);
   a.budget = budget;
+  return a;
+}
+
+// NVFP4: the scale-writer kernel; split-K partials are reduced in-kernel.
+cudaError_t run_fp4(const uint8_t* xq, const uint8_t* xs, const float* xg, const uint8_t* wq, const uint8_t* ws,
+                    const float* wg, const void* residual, void* Y, int64_t M, int64_t N, int64_t K,
+                    void* workspace, const GemmPlan& plan, long long budget, cudaStream_t s) {
+  const int64_t pitch = nvfp4_code_pitch(K);
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, xq, static_cast<uint64_t>(pitch), static_cast<uint64_t>(M), static_cast<uint64_t>(pitch), kBM) ||
+      !make_map(&tb, wq, static_cast<uint64_t>(pitch), static_cast<uint64_t>(N), static_cast<uint64_t>(pitch),
+                SfwCfg::BN))
+    return cudaErrorInvalidValue;
+  const GemmArgs a = make_args(true, SfwCfg::BN, xs, xg, ws, wg, residual, Y, M, N, K, workspace, plan, budget);
   const int grid = plan.grid < a.units ? plan.grid : a.units;
-  cudaError_t e;
-  if (FP4 && BN == 256) {
-    // tile counters: the first bytes of the workspace (zero between calls)
-    if (plan.splits > 1) a.counters = static_cast<unsigned int*>(workspace);
-    e = cudaFuncSetAttribute(gemm_fp4_sfw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SfwCfg::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    // split-K partials are reduced inside the kernel
-    return launch_pdl(gemm_fp4_sfw_kernel, dim3(grid), dim3(SfwCfg::THREADS), SfwCfg::SMEM_BYTES, s, ta, tb, a);
-  } else {
-    auto kern = gemm_kernel<FP4, BN>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, s, ta, tb, a);
-  }
+  cudaError_t e =
+      cudaFuncSetAttribute(gemm_fp4_sfw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SfwCfg::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(gemm_fp4_sfw_kernel, dim3(grid), dim3(SfwCfg::THREADS), SfwCfg::SMEM_BYTES, s, ta, tb, a);
+}
+
+// FP8: gemm_fp8_kernel<BN>, then the ordered split-K reduction when split.
+template <int BN>
+cudaError_t run_fp8(const uint8_t* xq, const float* xg, const uint8_t* wq, const float* wg, const void* residual,
+                    void* Y, int64_t M, int64_t N, int64_t K, void* workspace, const GemmPlan& plan,
+                    long long budget, cudaStream_t s) {
+  using C = Fp8Cfg<BN>;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(K), kBM) ||
+      !make_map(&tb, wq, static_cast<uint64_t>(K), static_cast<uint64_t>(N), static_cast<uint64_t>(K), BN))
+    return cudaErrorInvalidValue;
+  const GemmArgs a = make_args(false, BN, nullptr, xg, nullptr, wg, residual, Y, M, N, K, workspace, plan, budget);
+  const int grid = plan.grid < a.units ? plan.grid : a.units;
+  auto kern = gemm_fp8_kernel<BN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, s, ta, tb, a);
   if (e != cudaSuccess || plan.splits == 1) return e;
   const int64_t total8 = M * N / 8;
   const int threads = 256;
   const int64_t blocks = (total8 + threads - 1) / threads;
-  return launch_pdl(splitk_reduce_kernel<FP4>, dim3(static_cast<unsigned int>(blocks)), dim3(threads), 0, s,
+  return launch_pdl(splitk_reduce_kernel<false>, dim3(static_cast<unsigned int>(blocks)), dim3(threads), 0, s,
                     static_cast<const float*>(a.partial), plan.splits, a.M, a.N, xg, wg,
                     static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(Y));
 }
@@ -1011,12 +985,9 @@ cudaError_t launch_linear(bool fp4, const uint8_t* xq, const uint8_t* xs, const 
                           int64_t K, void* workspace, size_t ws_bytes, const GemmPlan& plan, long long budget,
                           cudaStream_t s) {
   (void)ws_bytes;
-  if (plan.bn == 256) {
-    if (fp4) return run<true, 256>(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
-    return run<false, 256>(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
-  }
-  if (fp4) return run<true, 128>(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
-  return run<false, 128>(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
+  if (fp4) return run_fp4(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
+  if (plan.bn == 256) return run_fp8<256>(xq, xg, wq, wg, residual, Y, M, N, K, workspace, plan, budget, s);
+  return run_fp8<128>(xq, xg, wq, wg, residual, Y, M, N, K, workspace, plan, budget, s);
 }
 
 cudaError_t read_and_clear_status(unsigned int* out, cudaStream_t s) {

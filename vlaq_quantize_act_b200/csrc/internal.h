@@ -68,6 +68,7 @@ cudaError_t launch_linear(bool fp4, const uint8_t* xq, const uint8_t* xs, const 
 // Device status word accessors (gemm.cu, quant.cu).
 cudaError_t read_and_clear_status(unsigned int* out, cudaStream_t s);
 cudaError_t read_and_clear_quant_status(unsigned int* out, cudaStream_t s);
+cudaError_t launch_selftest_wait_timeout(cudaStream_t s);
 
 // Kernel launch with the programmatic-stream-serialization attribute, so the
 // kernel may start while the previous kernel on the stream drains; every

@@ -144,13 +144,6 @@ __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t adesc, uint
       : "memory");
 }
 
-// Copy 32 rows x 16 bytes from shared memory into 32 TMEM lanes x 4
-// columns, replicated into all four 32-lane sub-partitions.
-__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
-}
-
 // 32 lanes x 4 consecutive 32-bit columns from registers: thread i writes
 // lane (base + i).  Completion is awaited with tmem_st_wait().
 __device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint4& v) {
@@ -223,17 +216,6 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
   d |= static_cast<uint64_t>(1024u >> 4) << 32;         // stride offset: 8 rows
   d |= static_cast<uint64_t>(1u) << 46;                 // descriptor version (sm_100)
   d |= static_cast<uint64_t>(2u) << 61;                 // 128-byte swizzle
-  return d;
-}
-
-// Descriptor of a 32-row x 16-byte block stored contiguously (no swizzle),
-// the source of tcgen05.cp 32x128b.
-__device__ __forceinline__ uint64_t sdesc_sf_block(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>(128u >> 4) << 16;          // leading offset (one 16-byte column)
-  d |= static_cast<uint64_t>(128u >> 4) << 32;          // stride offset: 8 rows x 16 B
-  d |= static_cast<uint64_t>(1u) << 46;
   return d;
 }
 

@@ -553,6 +553,25 @@ cudaError_t launch_scales_to_rowmajor(const uint8_t* in, uint8_t* out, int64_t r
                     dim3(threads), 0, s, in, out, rows, cols, nblk64);
 }
 
+namespace {
+// Failure-path self test: a bounded wait on an mbarrier that nothing ever
+// arrives on runs out and records the timeout like any library kernel.
+__global__ void selftest_wait_kernel(long long budget) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, budget)) atomicOr(&g_vlaq_quant_status, kStatusTimeout);
+}
+}  // namespace
+
+cudaError_t launch_selftest_wait_timeout(cudaStream_t s) {
+  selftest_wait_kernel<<<1, 32, 0, s>>>(2000000LL);  // about 1 ms of SM clock
+  return cudaGetLastError();
+}
+
 cudaError_t read_and_clear_quant_status(unsigned int* out, cudaStream_t s) {
   cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_vlaq_quant_status, sizeof(unsigned int), 0,
                                             cudaMemcpyDeviceToHost, s);
