@@ -57,6 +57,9 @@ def _load():
     lib.vo_transform_row_smooth.argtypes = [P, i64, P, ctypes.c_float, ctypes.c_uint, P, P]
     lib.vo_quantize_nvfp4_smooth.restype = ctypes.c_int
     lib.vo_quantize_nvfp4_smooth.argtypes = [P, i64, i64, P, ctypes.c_float, ctypes.c_uint, P, P, P, P]
+    lib.vo_quantize_nvfp4_static.restype = ctypes.c_int
+    lib.vo_quantize_nvfp4_static.argtypes = [P, i64, i64, P, ctypes.c_float, ctypes.c_uint, P, ctypes.c_float,
+                                             P, P, P]
     lib.vo_quantize_nvfp4.restype = ctypes.c_int
     lib.vo_quantize_nvfp4.argtypes = [P, i64, i64, P, ctypes.c_float, ctypes.c_uint,
                                       ctypes.c_int, P, P, P]
@@ -172,6 +175,24 @@ def quantize_nvfp4_smooth(X_bf16, smooth_f32, gamma_bf16=None, eps=1e-6, flags=0
                                           _ptr(codes), _ptr(scales), _ptr(g))
     if rc != 0:
         raise ValueError(f"oracle refused smoothed NVFP4 quantization of K={K} flags={flags}")
+    return codes, scales, g
+
+
+def quantize_nvfp4_static(X_bf16, g_static, smooth_f32=None, gamma_bf16=None, eps=1e-6, flags=0):
+    """Activations with a static global scale g_static (fp32) for every row;
+    optional per-channel smoothing.  Returns (codes, scales, g) as
+    quantize_nvfp4 (g = g_static per row)."""
+    X = _c(X_bf16, np.uint16)
+    rows, K = X.shape
+    a = None if smooth_f32 is None else _c(smooth_f32, np.float32)
+    g_in = None if gamma_bf16 is None else _c(gamma_bf16, np.uint16)
+    codes = np.zeros((rows, K // 2), dtype=np.uint8)
+    scales = np.zeros((rows, max(K // 16, 1)), dtype=np.uint8)
+    g = np.zeros(rows, dtype=np.float32)
+    rc = _load().vo_quantize_nvfp4_static(_ptr(X), rows, K, _ptr(g_in), ctypes.c_float(eps), flags, _ptr(a),
+                                          ctypes.c_float(g_static), _ptr(codes), _ptr(scales), _ptr(g))
+    if rc != 0:
+        raise ValueError(f"oracle refused static NVFP4 quantization of K={K} flags={flags}")
     return codes, scales, g
 
 

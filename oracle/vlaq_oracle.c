@@ -274,14 +274,14 @@ static void quant_block16(const float* y, int n, float g, uint8_t* sb8_out,
  * flag) or a gamma is missing for RMSNorm.
  */
 static int quantize_nvfp4(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* gamma, float eps,
-                          unsigned flags, const float* smooth, int per_tensor, uint8_t* codes, uint8_t* scales,
-                          float* g);
+                          unsigned flags, const float* smooth, int per_tensor, const float* g_static,
+                          uint8_t* codes, uint8_t* scales, float* g);
 
 int vo_quantize_nvfp4(const uint16_t* X, int64_t rows, int64_t K,
                       const uint16_t* gamma, float eps, unsigned flags,
                       int per_tensor, uint8_t* codes, uint8_t* scales,
                       float* g) {
-  return quantize_nvfp4(X, rows, K, gamma, eps, flags, NULL, per_tensor, codes, scales, g);
+  return quantize_nvfp4(X, rows, K, gamma, eps, flags, NULL, per_tensor, NULL, codes, scales, g);
 }
 
 /* Per-token NVFP4 quantization of activations smoothed per input channel
@@ -289,12 +289,25 @@ int vo_quantize_nvfp4(const uint16_t* X, int64_t rows, int64_t K,
 int vo_quantize_nvfp4_smooth(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* gamma, float eps,
                              unsigned flags, const float* smooth, uint8_t* codes, uint8_t* scales, float* g) {
   if (smooth == NULL) return -1;
-  return quantize_nvfp4(X, rows, K, gamma, eps, flags, smooth, 0, codes, scales, g);
+  return quantize_nvfp4(X, rows, K, gamma, eps, flags, smooth, 0, NULL, codes, scales, g);
+}
+
+/* Activations with a static (calibrated) global scale instead of the
+ * per-token amax: the ModelOpt / TensorRT NVFP4 linear carries an fp32
+ * input_scale ("NVIDIA/TensorRT-Edge-LLM PR #193", the pre_quant_scale
+ * commit lists weight, weight_scale, weight_scale_2 and input_scale).  Every
+ * row uses g = g_static; blocks and codes follow the same definitions, so
+ * values beyond the calibrated range saturate (E4M3 at 448, E2M1 at 6).  g
+ * receives g_static per row.  smooth may be NULL. */
+int vo_quantize_nvfp4_static(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* gamma, float eps,
+                             unsigned flags, const float* smooth, float g_static, uint8_t* codes,
+                             uint8_t* scales, float* g) {
+  return quantize_nvfp4(X, rows, K, gamma, eps, flags, smooth, 0, &g_static, codes, scales, g);
 }
 
 static int quantize_nvfp4(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* gamma, float eps,
-                          unsigned flags, const float* smooth, int per_tensor, uint8_t* codes, uint8_t* scales,
-                          float* g) {
+                          unsigned flags, const float* smooth, int per_tensor, const float* g_static,
+                          uint8_t* codes, uint8_t* scales, float* g) {
   if (K <= 0 || K % 16 != 0) return -1;
   if ((flags & VO_F_HADAMARD64) && K % 64 != 0) return -1;
   if ((flags & VO_F_RMSNORM) && gamma == NULL) return -1;
@@ -311,7 +324,10 @@ static int quantize_nvfp4(const uint16_t* X, int64_t rows, int64_t K, const uint
   for (int64_t r = 0; r < rows; ++r) {
     const float* y = Y + r * K;
     float gr = gt;
-    if (!per_tensor) {
+    if (g_static) {
+      gr = *g_static;
+      g[r] = gr;
+    } else if (!per_tensor) {
       float A = 0.0f;
       for (int64_t k = 0; k < K; ++k) A = fmaxf(A, fabsf(y[k]));
       gr = vo_nvfp4_global(A);

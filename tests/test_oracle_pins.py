@@ -461,3 +461,79 @@ def test_unit_smoothing_is_identity():
         got = oracle.quantize_nvfp4_smooth(bits(X), np.ones(320, np.float32), flags=fl)
         want = oracle.quantize_nvfp4(bits(X))
         assert all(np.array_equal(u, v) for u, v in zip(got, want))
+
+
+# ------------------------------------------------------------ static scale
+# A calibrated activation global scale (ModelOpt / TensorRT input_scale,
+# "NVIDIA/TensorRT-Edge-LLM PR #193") replaces the per-token amax; the block
+# and code definitions are unchanged.  The dynamic path is pinned above, so
+# equality with it at g = the row's own g transfers those pins; saturation
+# and underflow are checked against the E4M3 / E2M1 definitions in fp64.
+
+@pytest.mark.parametrize("flags,smoothed", [(0, False), (3, False), (2 | 8, True), (1 | 2 | 4, True)])
+def test_static_g_equal_to_row_g_reproduces_dynamic(flags, smoothed):
+    X = si.projection_activations(320, 7, 21)
+    gam = si.norm_gain(320, 21)
+    a = np.exp(np.random.default_rng(22).normal(0, 0.7, 320)).astype(np.float32) if smoothed else None
+    if smoothed:
+        c, s, g = oracle.quantize_nvfp4_smooth(bits(X), a, bits(gam), 1e-6, flags)
+    else:
+        c, s, g = oracle.quantize_nvfp4(bits(X), bits(gam), 1e-6, flags)
+    for r in range(7):
+        cs, ss, gs = oracle.quantize_nvfp4_static(bits(X)[r:r + 1], float(g[r]), a, bits(gam), 1e-6, flags)
+        assert np.array_equal(cs[0], c[r]) and np.array_equal(ss[0], s[r]) and gs[0] == g[r]
+
+
+def _static_check(y, codes, scales, g):
+    """Block scale = E4M3(max|y| / 6 g) (saturating at 448), code =
+    E2M1(y / S) with S = scale x g, checked in fp64 away from ties."""
+    K = y.size
+    for b in range(K // 16):
+        blk = y[16 * b:16 * b + 16].astype(np.float64)
+        q = np.abs(blk).max() / (6.0 * g)
+        sb = scales[b]
+        if q >= 464.0:
+            assert sb == 0x7E
+        elif q < 2.0 ** -10:
+            assert sb == 0
+        else:
+            assert abs(oracle.e4m3_decode(sb) - q) <= q * 2.0 ** -4 + 2.0 ** -10
+        S = oracle.e4m3_decode(sb) * g
+        for i in range(16):
+            c = (codes[8 * b + i // 2] >> (4 * (i % 2))) & 0xF
+            if S == 0:
+                assert c == 0
+                continue
+            v = blk[i] / S
+            if abs(v) > 5.0 * (1 + 1e-6):
+                assert c & 7 == 7 and (c >> 3) == (blk[i] < 0)
+            elif abs(v) <= 5.0 * (1 - 1e-6):
+                assert abs(abs(oracle.e2m1_decode(c)) - abs(v)) <= _grid_half_step(v) * (1 + 1e-6) + 1e-9
+
+
+@pytest.mark.parametrize("ratio", [1e-3, 0.3, 2.0, 1e3, 1e6])
+def test_static_saturation_and_rounding_definitions(ratio):
+    """g well below the row's own g (values beyond the calibrated range:
+    scales saturate at 448, codes at 6) and well above it (small block
+    scales, down to E4M3 zero and all-zero codes)."""
+    X = si.projection_activations(256, 5, 23)
+    xf = (bits(X).astype(np.uint32) << 16).view(np.float32)
+    _, _, gd = oracle.quantize_nvfp4(bits(X))
+    g = float(np.float32(gd.max() * ratio))
+    c, s, gs = oracle.quantize_nvfp4_static(bits(X), g)
+    assert np.all(gs == np.float32(g))
+    for r in range(5):
+        _static_check(xf[r], c[r], s[r], np.float32(g))
+    if ratio <= 1e-3:
+        assert (s == 0x7E).mean() > 0.5
+    if ratio >= 1e6:
+        assert (s == 0).any() and not c[s.repeat(8, axis=1) == 0].any()
+
+
+def test_static_extreme_scales_saturate_or_vanish():
+    X = si.projection_activations(64, 3, 24)
+    c, s, _ = oracle.quantize_nvfp4_static(bits(X), 1e-30)
+    nz = np.abs((bits(X).astype(np.uint32) << 16).view(np.float32)).reshape(3, 4, 16).max(axis=2) > 0
+    assert np.all(s[nz] == 0x7E)
+    c, s, _ = oracle.quantize_nvfp4_static(bits(X), 1e38)   # 6 g overflows: every block scale 0
+    assert not s.any() and not c.any()
