@@ -69,6 +69,12 @@ def _load():
     lib.vo_quantize_fp8.argtypes = [P, i64, i64, P, ctypes.c_float, ctypes.c_uint, P, P]
     lib.vo_decode_fp8.restype = None
     lib.vo_decode_fp8.argtypes = [P, P, i64, i64, P]
+    lib.vo_quantize_int8.restype = ctypes.c_int
+    lib.vo_quantize_int8.argtypes = [P, i64, i64, P, ctypes.c_float, ctypes.c_uint, P, P]
+    lib.vo_decode_int8.restype = None
+    lib.vo_decode_int8.argtypes = [P, P, i64, i64, P]
+    lib.vo_linear_int8.restype = None
+    lib.vo_linear_int8.argtypes = [P, P, P, P, P, i64, i64, i64, P, i64, P, P]
     lib.vo_linear_f64.restype = None
     lib.vo_linear_f64.argtypes = [P, P, P, i64, i64, i64, P, i64, P]
     lib.vo_num_threads.restype = ctypes.c_int
@@ -229,6 +235,48 @@ def decode_fp8(codes, s) -> np.ndarray:
     out = np.empty((rows, K), dtype=np.float64)
     _load().vo_decode_fp8(_ptr(codes), _ptr(s), rows, K, _ptr(out))
     return out
+
+
+# -------------------------------------------------------------------- INT8
+def quantize_int8(X_bf16, gamma_bf16=None, eps=1e-6, flags=0):
+    """Symmetric per-row INT8: returns (codes i8 [rows, K], s f32 [rows])."""
+    X = _c(X_bf16, np.uint16)
+    rows, K = X.shape
+    g_in = None if gamma_bf16 is None else _c(gamma_bf16, np.uint16)
+    codes = np.zeros((rows, K), dtype=np.int8)
+    s = np.zeros(rows, dtype=np.float32)
+    rc = _load().vo_quantize_int8(_ptr(X), rows, K, _ptr(g_in), ctypes.c_float(eps), flags, _ptr(codes), _ptr(s))
+    if rc != 0:
+        raise ValueError(f"oracle refused INT8 quantization of K={K} flags={flags}")
+    return codes, s
+
+
+def decode_int8(codes, s) -> np.ndarray:
+    codes = _c(codes, np.int8)
+    s = _c(s, np.float32)
+    rows, K = codes.shape
+    out = np.empty((rows, K), dtype=np.float64)
+    _load().vo_decode_int8(_ptr(codes), _ptr(s), rows, K, _ptr(out))
+    return out
+
+
+def linear_int8(cx, sx, cw, sw, residual_bf16=None, rows=None):
+    """INT8 GEMM + epilogue for the selected rows: returns (Y bf16 bits
+    uint16 [nrows, N], exact integer sums int64 [nrows, N])."""
+    cx = _c(cx, np.int8)
+    cw = _c(cw, np.int8)
+    sx = _c(sx, np.float32)
+    sw = _c(sw, np.float32)
+    M, K = cx.shape
+    N = cw.shape[0]
+    res = None if residual_bf16 is None else _c(residual_bf16, np.uint16)
+    idx = None if rows is None else _c(rows, np.int64)
+    nrows = M if rows is None else len(idx)
+    Y = np.zeros((nrows, N), dtype=np.uint16)
+    acc = np.zeros((nrows, N), dtype=np.int64)
+    _load().vo_linear_int8(_ptr(cx), _ptr(sx), _ptr(cw), _ptr(sw), _ptr(res), M, N, K, _ptr(idx), nrows, _ptr(Y),
+                           _ptr(acc))
+    return Y, acc
 
 
 # -------------------------------------------------------------------- GEMM

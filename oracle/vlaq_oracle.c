@@ -392,6 +392,82 @@ void vo_decode_fp8(const uint8_t* codes, const float* s, int64_t rows,
       out[r * K + k] = vo_e4m3_decode(codes[r * K + k]) * (double)s[r];
 }
 
+/* ---------------------------------------------------------------- INT8 -- */
+/*
+ * INT8 symmetric per-row quantization ("FoldQuant W8A8/W4A4 inference ...":
+ * INT8 codes with per-row weight scales, activations quantized per token;
+ * its OpenVINO commit lists per-token amax scale, round-half-even, clamp):
+ * s = max|y| / 127 (fp32), code = clamp(RNE(fp32(y / s)), -127, 127), or 0
+ * when s == 0.  Decoded value: code * s.
+ */
+static int8_t int8_code(float q) {
+  float r = nearbyintf(q); /* default rounding mode: half to even */
+  if (r > 127.0f) r = 127.0f;
+  if (r < -127.0f) r = -127.0f;
+  return (int8_t)r;
+}
+
+int vo_quantize_int8(const uint16_t* X, int64_t rows, int64_t K, const uint16_t* gamma, float eps,
+                     unsigned flags, int8_t* codes, float* s) {
+  if (K <= 0 || K % 16 != 0) return -1;
+  if ((flags & VO_F_HADAMARD64) && K % 64 != 0) return -1;
+  if ((flags & VO_F_RMSNORM) && gamma == NULL) return -1;
+  float* y = (float*)malloc(sizeof(float) * (size_t)K);
+  for (int64_t r = 0; r < rows; ++r) {
+    vo_transform_row(X + r * K, K, gamma, eps, flags, y);
+    float A = 0.0f;
+    for (int64_t k = 0; k < K; ++k) A = fmaxf(A, fabsf(y[k]));
+    float sr = A / 127.0f;
+    s[r] = sr;
+    for (int64_t k = 0; k < K; ++k) codes[r * K + k] = (sr == 0.0f) ? 0 : int8_code(y[k] / sr);
+  }
+  free(y);
+  return 0;
+}
+
+void vo_decode_int8(const int8_t* codes, const float* s, int64_t rows, int64_t K, double* out) {
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t k = 0; k < K; ++k) out[r * K + k] = (double)codes[r * K + k] * (double)s[r];
+}
+
+/* fp32 -> bf16, round to nearest even on the bit pattern (finite inputs). */
+static uint16_t f32_to_bf16_rne(float v) {
+  uint32_t u;
+  memcpy(&u, &v, 4);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+/*
+ * INT8 GEMM and its epilogue.  The integer sum is exact in any order (the
+ * FoldQuant SYCL commit relies on that), so the output has one value:
+ * acc = sum_k cx[m, k] cw[n, k] (int64), t = fp32(acc), c = fp32(s_x[m]
+ * s_w[n]), y = fp32(t c), y = fp32(y + residual[m, n]) when a residual is
+ * given, out = bf16(y) (round to nearest even).  Rows row_idx (all M when
+ * NULL; nrows must then equal M).  acc_out (int64 [nrows, N]) may be NULL.
+ */
+void vo_linear_int8(const int8_t* cx, const float* sx, const int8_t* cw, const float* sw, const uint16_t* residual,
+                    int64_t M, int64_t N, int64_t K, const int64_t* row_idx, int64_t nrows, uint16_t* Y,
+                    int64_t* acc_out) {
+  (void)M;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t i = 0; i < nrows; ++i) {
+    int64_t m = row_idx ? row_idx[i] : i;
+    const int8_t* x = cx + m * K;
+    for (int64_t n = 0; n < N; ++n) {
+      const int8_t* w = cw + n * K;
+      int64_t acc = 0;
+      for (int64_t k = 0; k < K; ++k) acc += (int64_t)x[k] * (int64_t)w[k];
+      if (acc_out) acc_out[i * N + n] = acc;
+      float t = (float)acc;
+      float c = sx[m] * sw[n];
+      float y = t * c;
+      if (residual) y = y + vo_bf16_to_f32(residual[m * N + n]);
+      Y[i * N + n] = f32_to_bf16_rne(y);
+    }
+  }
+}
+
 /* ---------------------------------------------------------------- GEMM -- */
 /*
  * Y[i, n] = sum_k Xd[row_i, k] * Wd[n, k] + residual[row_i, n], fp64, k in

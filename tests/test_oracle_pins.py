@@ -537,3 +537,118 @@ def test_static_extreme_scales_saturate_or_vanish():
     assert np.all(s[nz] == 0x7E)
     c, s, _ = oracle.quantize_nvfp4_static(bits(X), 1e38)   # 6 g overflows: every block scale 0
     assert not s.any() and not c.any()
+
+
+# ------------------------------------------------------------------- INT8
+# Symmetric per-row INT8 ("FoldQuant W8A8/W4A4 inference ...": per-row
+# weight scales, per-token activations, round-half-even, clamp) and the
+# exact integer GEMM with its fp32 epilogue.
+
+def test_int8_ties_golden():
+    rows = list(_golden_lines("int8_ties.txt"))
+    x = [float(r[0]) for r in rows]
+    want = np.array([int(r[1]) for r in rows], np.int8)
+    K = 32
+    X = _bits_bf16(x + [0.0] * (K - len(x))).reshape(1, K)
+    codes, s = oracle.quantize_int8(X)
+    assert s[0] == np.float32(1.0)
+    assert np.array_equal(codes[0, :len(x)], want)
+
+
+def test_int8_error_bound_max_element_and_zero_row():
+    rng = np.random.default_rng(31)
+    rows, K = 12, 320
+    X = (rng.standard_normal((rows, K)) * np.exp(rng.standard_normal(K))).astype(np.float32)
+    X[2] = 0.0
+    X[5, 9] = -3e3
+    Xb = _bits_bf16(X.ravel()).reshape(rows, K)
+    xf = (Xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    codes, s = oracle.quantize_int8(Xb)
+    deq = oracle.decode_int8(codes, s)
+    for r in range(rows):
+        A = np.abs(xf[r]).max()
+        if A == 0:
+            assert s[r] == 0 and not codes[r].any()
+            continue
+        assert abs(float(s[r]) - A / 127) <= A / 127 * 2.0 ** -24
+        # half a step, plus the rounding of s and of the quotient
+        assert np.all(np.abs(xf[r] - deq[r]) <= float(s[r]) * (0.5 + 1e-5))
+        j = int(np.argmax(np.abs(xf[r])))
+        assert abs(int(codes[r, j])) == 127 and np.sign(codes[r, j]) == np.sign(xf[r, j])
+        assert codes[r].min() >= -127
+
+
+def test_int8_power_of_two_scale_invariance():
+    X = si.projection_activations(256, 4, 32)
+    xf = (bits(X).astype(np.uint32) << 16).view(np.float32)
+    c0, s0 = oracle.quantize_int8(bits(X))
+    for k in (-40, -1, 7, 60):
+        c1, s1 = oracle.quantize_int8(_bits_bf16((xf.astype(np.float64) * 2.0 ** k).ravel()).reshape(xf.shape))
+        assert np.array_equal(c0, c1)
+        assert np.array_equal(s1, (s0.astype(np.float64) * 2.0 ** k).astype(np.float32))
+
+
+def test_int8_gemm_integer_sums_equal_numpy():
+    rng = np.random.default_rng(33)
+    cx = rng.integers(-127, 128, (9, 200), dtype=np.int8)
+    cw = rng.integers(-127, 128, (24, 200), dtype=np.int8)
+    _, acc = oracle.linear_int8(cx, np.ones(9, np.float32), cw, np.ones(24, np.float32))
+    assert np.array_equal(acc, cx.astype(np.int64) @ cw.astype(np.int64).T)
+    # every product at the extreme: K * 127^2 (the int32 bound the kernel relies on)
+    K = 32768
+    _, acc = oracle.linear_int8(np.full((1, K), -127, np.int8), np.ones(1, np.float32),
+                                np.full((8, K), 127, np.int8), np.ones(8, np.float32))
+    assert np.all(acc == -K * 127 * 127) and K * 127 * 127 < 2 ** 31
+
+
+def test_int8_gemm_power_of_two_scales_are_exact_bf16_rounding():
+    """s_x, s_w powers of two and |acc| < 2^24: t, c and t c are exact, so
+    the output is torch's bf16 rounding of acc * s_x * s_w."""
+    rng = np.random.default_rng(34)
+    K = 512
+    cx = rng.integers(-127, 128, (6, K), dtype=np.int8)
+    cw = rng.integers(-127, 128, (16, K), dtype=np.int8)
+    sx = np.exp2(rng.integers(-20, 5, 6)).astype(np.float32)
+    sw = np.exp2(rng.integers(-20, 5, 16)).astype(np.float32)
+    Y, acc = oracle.linear_int8(cx, sx, cw, sw)
+    exact = acc.astype(np.float64) * sx[:, None].astype(np.float64) * sw[None, :].astype(np.float64)
+    want = torch.from_numpy(exact.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.all(np.abs(acc) < 2 ** 24) and np.array_equal(Y, want)
+
+
+def test_int8_gemm_residual_and_decode_identity():
+    """Against the fp64 product of the decoded operands (+ residual): within
+    the bf16 rounding of the output and the fp32 epilogue steps."""
+    X = si.projection_activations(448, 7, 35)
+    W = si.projection_weight(448, 40, 35)
+    R = torch.randn(7, 40, generator=torch.Generator().manual_seed(35)).to(torch.bfloat16)
+    cx, sx = oracle.quantize_int8(bits(X))
+    cw, sw = oracle.quantize_int8(bits(W))
+    Y, _ = oracle.linear_int8(cx, sx, cw, sw, bits(R))
+    ref = oracle.linear_f64(oracle.decode_int8(cx, sx), oracle.decode_int8(cw, sw), bits(R))
+    y = (Y.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert np.all(np.abs(y - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6 * np.abs(ref).max())
+
+
+def test_int8_brute_force_1x16x1():
+    """bf16 inputs -> codes -> product, against exact rationals: the code is
+    the nearest integer to y / s (ties even) and the output is within one
+    bf16 half-ulp (plus fp32 epilogue rounding) of the exact product."""
+    rng = np.random.default_rng(36)
+    for trial in range(20):
+        x = _bits_bf16((rng.standard_normal(16) * 3).astype(np.float32)).reshape(1, 16)
+        w = _bits_bf16((rng.standard_normal(16) * 0.1).astype(np.float32)).reshape(1, 16)
+        cx, sx = oracle.quantize_int8(x)
+        cw, sw = oracle.quantize_int8(w)
+        for v, c, s in ((x, cx, sx), (w, cw, sw)):
+            vf = (v.astype(np.uint32) << 16).view(np.float32)[0]
+            for i in range(16):
+                q = Fraction(float(vf[i])) / Fraction(float(s[0]))
+                lo = math.floor(q)
+                best = lo if (q - lo < Fraction(1, 2) or (q - lo == Fraction(1, 2) and lo % 2 == 0)) else lo + 1
+                # fp32 rounding of the quotient can only move an exact tie candidate by < 2^-17 relative
+                assert abs(int(c[0, i]) - best) <= (1 if abs(q - lo - Fraction(1, 2)) < abs(q) * 2 ** -22 else 0)
+        Y, acc = oracle.linear_int8(cx, sx, cw, sw)
+        exact = Fraction(int(acc[0, 0])) * Fraction(float(sx[0])) * Fraction(float(sw[0]))
+        y = float((Y.astype(np.uint32) << 16).view(np.float32)[0, 0])
+        assert abs(Fraction(y) - exact) <= abs(exact) * Fraction(1, 2 ** 8) * Fraction(1001, 1000)
