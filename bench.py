@@ -19,7 +19,8 @@ Reported (one JSON line on rank 0):
   prologue   the activation prologue: algorithmic bytes / duration vs HBM
   decode     M = 1 (weight-bandwidth-bound): GB/s of algorithmic bytes,
              weights rotated over two copies so the working set exceeds L2
-  fp8        the FP8 W8A8 variant of the same step (TFLOP/s)
+  fp8, int8  the FP8 and INT8 W8A8 variants of the same step (TFLOP/s; INT8
+             multiply-accumulates counted as FLOPs)
   cpu_baseline  the CPU oracle on a bounded sample of the same workload
 Inputs: seeded synthetic bf16 (synthetic_inputs.py); the per-step working set
 (X 61 MB + W 131 MB + Y 102 MB) exceeds the 126 MB L2.
@@ -165,19 +166,25 @@ def make_inputs(M, device, seed_offset=0):
 class Step:
     """Device buffers and launch sequence of one hot-path step."""
 
-    def __init__(self, vq, data, M, device, fp8=False, weight_copies=1):
+    def __init__(self, vq, data, M, device, fmt="nvfp4", weight_copies=1):
+        assert fmt in ("nvfp4", "fp8", "int8"), fmt
         self.vq = vq
         self.M = M
-        self.fp8 = fp8
+        self.fmt = fmt
+        self.fp8 = fmt != "nvfp4"  # an 8-bit W8A8 format (FP8 or INT8)
         self.layers = []
         for name in PROJ:
             K, N, X, W = data[name]
             Wd = W.to(device)
             copies = []
             for _ in range(weight_copies):
-                if fp8:
+                if fmt == "fp8":
                     wq, sw = vq.alloc_fp8(N, K, device)
                     vq.vlaq_quantize_weight_fp8(Wd, N, K, 0, wq, sw)
+                    copies.append((wq, None, sw))
+                elif fmt == "int8":
+                    wq, sw = vq.alloc_int8(N, K, device)
+                    vq.vlaq_quantize_weight_int8(Wd, N, K, 0, wq, sw)
                     copies.append((wq, None, sw))
                 else:
                     wq, ws, wg = vq.alloc_nvfp4(N, K, device, per_tensor=True)
@@ -185,8 +192,8 @@ class Step:
                     copies.append((wq, ws, wg))
             del Wd
             Xd = X.to(device)
-            if fp8:
-                xq, sx = vq.alloc_fp8(M, K, device)
+            if self.fp8:
+                xq, sx = (vq.alloc_fp8 if fmt == "fp8" else vq.alloc_int8)(M, K, device)
                 act = (xq, None, sx)
             else:
                 act = vq.alloc_nvfp4(M, K, device)
@@ -205,14 +212,18 @@ class Step:
             wq, ws, wg = L["W"][copy % len(L["W"])]
             if events is not None:
                 events[i][0].record()
-            if self.fp8:
+            if self.fmt == "fp8":
                 vq.vlaq_quantize_act_fp8(L["X"], M, K, None, 1e-6, 0, xq, xg)
+            elif self.fmt == "int8":
+                vq.vlaq_quantize_act_int8(L["X"], M, K, None, 1e-6, 0, xq, xg)
             else:
                 vq.vlaq_quantize_act_nvfp4(L["X"], M, K, None, 1e-6, 0, xq, xs, xg)
             if events is not None:
                 events[i][1].record()
-            if self.fp8:
+            if self.fmt == "fp8":
                 vq.vlaq_linear_fp8(xq, xg, wq, wg, None, L["Y"], M, N, K, L["ws"], L["nb"])
+            elif self.fmt == "int8":
+                vq.vlaq_linear_int8(xq, xg, wq, wg, None, L["Y"], M, N, K, L["ws"], L["nb"])
             else:
                 vq.vlaq_linear_nvfp4(xq, xs, xg, wq, ws, wg, None, L["Y"], M, N, K, L["ws"], L["nb"])
             if events is not None:
@@ -232,53 +243,73 @@ class Step:
         return M * K * 2 + M * K // 2 + M * K // 16 + 4 * M
 
 
-def stack_weights(vq, device, layers=si.STACK_LAYERS):
-    """NVFP4 weights of the 28-layer stack in (layer, projection) order, each
-    quantized on the device right after it is generated (only the NVFP4 copy
-    stays: about 3.7 GB)."""
+# the mixed-precision stack: these projections in FP8 W8A8, the rest NVFP4
+MIXED_FP8 = ("o", "down")
+
+
+def stack_weights(vq, device, layers=si.STACK_LAYERS, fp8=()):
+    """Weights of the 28-layer stack in (layer, projection) order, each
+    quantized on the device right after it is generated (only the quantized
+    copy stays: about 3.7 GB all NVFP4).  Projections named in fp8 get FP8
+    codes and per-row scales (2-tuples), the others NVFP4 (3-tuples)."""
     out = []
     for l in range(layers):
         for p, (name, K, N) in enumerate(si.STACK_PROJECTIONS):
             W = si.projection_weight(K, N, si.stack_seed(l, p)).to(device)
-            wq, ws, wg = vq.alloc_nvfp4(N, K, device, per_tensor=True)
-            vq.vlaq_quantize_weight_nvfp4(W, N, K, 0, wq, ws, wg)
+            if name in fp8:
+                wq, sw = vq.alloc_fp8(N, K, device)
+                vq.vlaq_quantize_weight_fp8(W, N, K, 0, wq, sw)
+                out.append((wq, sw))
+            else:
+                wq, ws, wg = vq.alloc_nvfp4(N, K, device, per_tensor=True)
+                vq.vlaq_quantize_weight_nvfp4(W, N, K, 0, wq, ws, wg)
+                out.append((wq, ws, wg))
             del W
-            out.append((wq, ws, wg))
     torch.cuda.synchronize()
     return out
 
 
 class Stack:
-    """The 28-layer stack of seven unfused projections (196 NVFP4 GEMMs):
-    every (layer, projection) has its own seeded weight and its own seeded
-    activations [M, K]; run() is one prologue + GEMM per entry."""
+    """The 28-layer stack of seven unfused projections (196 GEMMs): every
+    (layer, projection) has its own seeded weight and its own seeded
+    activations [M, K]; run() is one prologue + GEMM per entry.  All NVFP4
+    by default; with fp8 = MIXED_FP8 the o and down projections run FP8
+    W8A8 (per-row scales) and q/k/v/gate/up NVFP4."""
 
-    def __init__(self, vq, M, device, layers=si.STACK_LAYERS, weights=None):
+    def __init__(self, vq, M, device, layers=si.STACK_LAYERS, weights=None, fp8=()):
         self.vq = vq
         self.M = M
         self.entries = []
         if weights is None:
-            weights = stack_weights(vq, device, layers)
+            weights = stack_weights(vq, device, layers, fp8)
         for l in range(layers):
             for p, (name, K, N) in enumerate(si.STACK_PROJECTIONS):
                 seed = si.stack_seed(l, p)
-                wq, ws, wg = weights[7 * l + p]
+                W = weights[7 * l + p]
+                is8 = name in fp8
+                assert len(W) == (2 if is8 else 3), (name, len(W))
                 X = si.projection_activations(K, M, seed).to(device)
                 wsp, nb = vq.alloc_workspace(M, N, K, device)
-                self.entries.append(dict(layer=l, proj=p, name=name, K=K, N=N, W=(wq, ws, wg), X=X,
-                                         act=vq.alloc_nvfp4(M, K, device),
+                act = vq.alloc_fp8(M, K, device) if is8 else vq.alloc_nvfp4(M, K, device)
+                self.entries.append(dict(layer=l, proj=p, name=name, K=K, N=N, W=W, X=X, fp8=is8, act=act,
                                          Y=torch.empty(M, N, dtype=torch.bfloat16, device=device), ws=wsp, nb=nb))
         torch.cuda.synchronize()
         self.flops = sum(2.0 * M * e["N"] * e["K"] for e in self.entries)
-        self.weight_bytes = sum(e["W"][0].numel() + e["W"][1].numel() + 4 for e in self.entries)
+        self.weight_bytes = sum(sum(t.numel() * t.element_size() for t in e["W"]) for e in self.entries)
 
     def run(self, copy=0):
         vq, M = self.vq, self.M
         for e in self.entries:
-            xq, xs, xg = e["act"]
-            wq, ws, wg = e["W"]
-            vq.vlaq_quantize_act_nvfp4(e["X"], M, e["K"], None, 1e-6, 0, xq, xs, xg)
-            vq.vlaq_linear_nvfp4(xq, xs, xg, wq, ws, wg, None, e["Y"], M, e["N"], e["K"], e["ws"], e["nb"])
+            if e["fp8"]:
+                xq, sx = e["act"]
+                wq, sw = e["W"]
+                vq.vlaq_quantize_act_fp8(e["X"], M, e["K"], None, 1e-6, 0, xq, sx)
+                vq.vlaq_linear_fp8(xq, sx, wq, sw, None, e["Y"], M, e["N"], e["K"], e["ws"], e["nb"])
+            else:
+                xq, xs, xg = e["act"]
+                wq, ws, wg = e["W"]
+                vq.vlaq_quantize_act_nvfp4(e["X"], M, e["K"], None, 1e-6, 0, xq, xs, xg)
+                vq.vlaq_linear_nvfp4(xq, xs, xg, wq, ws, wg, None, e["Y"], M, e["N"], e["K"], e["ws"], e["nb"])
 
 
 def capture(step, copies=1):
@@ -590,19 +621,21 @@ def main():
                                                     for i, L in enumerate(dstep.layers)}}
         del dstep, dgraph
 
-        # ---------------- FP8 W8A8 variant of the prefill step
-        fstep = Step(vq, data, M_PREFILL, device, fp8=True)
-        fgraph = capture(fstep)
-        for _ in range(args.warmup):
-            fgraph.replay()
-        fms = time_graph(fgraph, args.steps, dist_on, device)
-        _, fgem, _ = kernel_durations(fstep, max(args.steps // 2, 3))
-        fgem_ms = sum(sum(x) for x in fgem) / len(fgem[0])
-        fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
-        out["fp8"] = {"value": world * fstep.flops / (fms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": fms,
-                      "gemm_achieved": fstep.flops / (fgem_ms / 1e3) / 1e12, "peak": fp8_peak,
-                      "frac": fstep.flops / (fgem_ms / 1e3) / 1e12 / fp8_peak}
-        del fstep, fgraph
+        # ---------------- FP8 and INT8 W8A8 variants of the prefill step (the
+        # dense 8-bit tensor-core rate is twice bf16 for both kinds)
+        for fmt in ("fp8", "int8"):
+            fstep = Step(vq, data, M_PREFILL, device, fmt=fmt)
+            fgraph = capture(fstep)
+            for _ in range(args.warmup):
+                fgraph.replay()
+            fms = time_graph(fgraph, args.steps, dist_on, device)
+            _, fgem, _ = kernel_durations(fstep, max(args.steps // 2, 3))
+            fgem_ms = sum(sum(x) for x in fgem) / len(fgem[0])
+            fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
+            out[fmt] = {"value": world * fstep.flops / (fms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": fms,
+                        "gemm_achieved": fstep.flops / (fgem_ms / 1e3) / 1e12, "peak": fp8_peak,
+                        "frac": fstep.flops / (fgem_ms / 1e3) / 1e12 / fp8_peak}
+            del fstep, fgraph
 
         # ---------------- e2e through the public API with host buffers
         hostX = [L["X"].cpu().pin_memory() for L in step.layers]
@@ -635,9 +668,12 @@ def main():
     if not args.quick:
         # ---------------- prologue variants over the four projection inputs:
         # fused RMSNorm + block-64 rotation, per-channel smoothing (divide,
-        # before the rotation), and both; same bytes as the plain prologue
-        # (the gains and smoothing factors stay in cache)
-        variants = {"fused_rmsnorm_wht": (3, False), "smooth": (0, True), "fused_smooth": (3, True)}
+        # before the rotation), both, and a static calibrated global scale
+        # (no row-amax pass) plain and fused; same bytes as the plain
+        # prologue (the gains and smoothing factors stay in cache)
+        variants = {"fused_rmsnorm_wht": (3, False, None), "smooth": (0, True, None),
+                    "fused_smooth": (3, True, None), "static": (0, False, 0.01),
+                    "fused_static": (3, False, 0.01)}
         extra = {}
         for L in step.layers:
             K = L["K"]
@@ -646,13 +682,16 @@ def main():
                                 torch.from_numpy(np.exp(rng.uniform(np.log(0.1553), np.log(6.4375), K))
                                                  .astype(np.float32)).to(device))
         out["prologue_variants"] = {}
-        for vname, (vflags, vsmooth) in variants.items():
+        for vname, (vflags, vsmooth, vstatic) in variants.items():
             class _PV:
                 def run(self, c=0):
                     for L in step.layers:
                         xq, xs, xg = L["act"]
                         gam, sm = extra[L["name"]]
-                        if vsmooth:
+                        if vstatic is not None:
+                            vq.vlaq_quantize_act_nvfp4_static(L["X"], M_PREFILL, L["K"], gam, None, 1e-6, vflags,
+                                                              vstatic, xq, xs, xg)
+                        elif vsmooth:
                             vq.vlaq_quantize_act_nvfp4_smooth(L["X"], M_PREFILL, L["K"], gam, sm, 1e-6, vflags,
                                                               xq, xs, xg)
                         else:
@@ -691,23 +730,25 @@ def main():
 
     if args.stack:
         # ---------------- 28-layer stack: one graph of 196 prologue + GEMM pairs
+        # (all NVFP4, then mixed: o / down FP8 W8A8, the rest NVFP4)
         out["stack"] = {}
-        sw = stack_weights(vq, device)
-        for sm in (M_PREFILL, 1):
-            st = Stack(vq, sm, device, weights=sw)
-            sg = capture(st)
-            for _ in range(args.warmup):
-                sg.replay()
-            torch.cuda.synchronize()
-            sms = time_graph(sg, max(args.steps // 4, 3), dist_on, device)
-            key = "prefill" if sm > 1 else "decode"
-            out["stack"][key] = {"M": sm, "ms": sms, "us_per_token": 1e3 * sms / sm,
-                                 "tflops": world * st.flops / (sms / 1e3) / 1e12,
-                                 "weight_gbs": world * st.weight_bytes / (sms / 1e3) / 1e9,
-                                 "gemms": len(st.entries)}
-            del sg, st
-            torch.cuda.empty_cache()
-        del sw
+        for prefix, fp8 in (("", ()), ("mixed_", MIXED_FP8)):
+            sw = stack_weights(vq, device, fp8=fp8)
+            for sm in (M_PREFILL, 1):
+                st = Stack(vq, sm, device, weights=sw, fp8=fp8)
+                sg = capture(st)
+                for _ in range(args.warmup):
+                    sg.replay()
+                torch.cuda.synchronize()
+                sms = time_graph(sg, max(args.steps // 4, 3), dist_on, device)
+                key = prefix + ("prefill" if sm > 1 else "decode")
+                out["stack"][key] = {"M": sm, "ms": sms, "us_per_token": 1e3 * sms / sm,
+                                     "tflops": world * st.flops / (sms / 1e3) / 1e12,
+                                     "weight_gbs": world * st.weight_bytes / (sms / 1e3) / 1e9,
+                                     "gemms": len(st.entries), "fp8_projections": list(fp8)}
+                del sg, st
+                torch.cuda.empty_cache()
+            del sw
 
     # launches of our kernels inside the timed region: per step 4 prologues +
     # 4 GEMMs (+ split-K reductions when planned)

@@ -176,6 +176,28 @@ VLAQ_API vlaq_status vlaq_quantize_act_nvfp4_smooth(const void* X, int64_t M, in
                                             float eps, uint32_t flags, uint8_t* codes,
                                             uint8_t* scales, float* g_x, void* stream);
 
+/* vlaq_quantize_act_nvfp4 with a static (calibrated) global scale instead
+ * of the per-token amax: the fp32 input_scale that ModelOpt / TensorRT
+ * NVFP4 checkpoints store beside weight_scale and weight_scale_2
+ * ("NVIDIA/TensorRT-Edge-LLM PR #193", pre_quant_scale commit).  Every row
+ * uses g = g_static; block scales and codes follow the same definitions
+ * (block scale E4M3(max|y| / (6 g)), code E2M1(y / (E4M3 scale x g))), so
+ * values beyond the calibrated range saturate at scale 448 and code 6.
+ * g_x[m] receives g_static for every row, so vlaq_linear_nvfp4 consumes the
+ * result unchanged.  The row-amax pass and its reduction are skipped.
+ *   g_static  finite and > 0 (host value), else VLAQ_ERR_INVALID_ARG
+ *   smooth    fp32 [K] (device, 16-byte aligned) or NULL; required when a
+ *             smoothing flag is set (as vlaq_quantize_act_nvfp4_smooth)
+ *   flags     any of VLAQ_F_RMSNORM | VLAQ_F_HADAMARD64 | VLAQ_F_SMOOTH_AFTER
+ *             | VLAQ_F_SMOOTH_MUL (the smoothing flags only with smooth)
+ * Other arguments, outputs and limits as vlaq_quantize_act_nvfp4.  Finite
+ * inputs only. */
+VLAQ_API vlaq_status vlaq_quantize_act_nvfp4_static(const void* X, int64_t M, int64_t K,
+                                            const void* gamma, const float* smooth,
+                                            float eps, uint32_t flags, float g_static,
+                                            uint8_t* codes, uint8_t* scales, float* g_x,
+                                            void* stream);
+
 /* Block scales from the 128x4 tiled layout the GEMM reads (as written by
  * the NVFP4 quantizers, vlaq_nvfp4_scale_bytes(rows, K) bytes) to the
  * logical row-major layout: out[r * (K/16) + b] = E4M3 scale of row r,
@@ -188,10 +210,10 @@ VLAQ_API vlaq_status vlaq_quantize_act_nvfp4_smooth(const void* X, int64_t M, in
 VLAQ_API vlaq_status vlaq_scales_to_rowmajor(const uint8_t* in, uint8_t* out, int64_t rows, int64_t K,
                                              void* stream);
 
-/* Bytes of workspace vlaq_linear_nvfp4 / vlaq_linear_fp8 need for the given
+/* Bytes of workspace vlaq_linear_nvfp4 / _fp8 / _int8 need for the given
  * shape on the current device (0 when the shape runs without split-K).  The
  * workspace's first 1024 bytes hold vlaq_linear_nvfp4's per-tile arrival
- * counters, the per-split fp32 partial sums follow.  The counters must be
+ * counters, the per-split partial sums (fp32, s32 for INT8) follow.  The counters must be
  * zero when a call starts: zero the workspace once after allocating it;
  * every call (of any shape, NVFP4 or FP8) leaves them zero again, so nothing
  * is cleared between calls.  After vlaq_check reports VLAQ_ERR_TIMEOUT, zero
@@ -264,6 +286,42 @@ VLAQ_API vlaq_status vlaq_linear_fp8(const uint8_t* xq, const float* s_x,
                             const void* residual, void* Y, int64_t M,
                             int64_t N, int64_t K, void* workspace,
                             size_t ws_bytes, void* stream);
+
+/* ----------------------------------------------------------- INT8 W8A8 */
+/* FoldQuant's 8-bit integer path ("FoldQuant W8A8/W4A4 inference and
+ * FoldQuantVLA quantized-model converter", vla.cpp PR #33: INT8 codes with
+ * per-row weight scales, activations quantized per token; its OpenVINO
+ * commit: per-token amax scale, round-half-even, clamp).  Symmetric:
+ * s = max|y| / 127 (fp32, correctly rounded), code = clamp(RNE(y / s), -127,
+ * 127) with y / s correctly rounded in fp32; an all-zero row gets s = 0 and
+ * zero codes.  Codes are two's-complement int8, row-major [rows, K]. */
+
+/* Per-row weight quantization.  W bf16 [N, K]; flags 0 or
+ * VLAQ_F_HADAMARD64; codes out [N, K]; s_w out, N fp32.
+ * Limits: 16 <= K <= 32768, K % 16 == 0. */
+VLAQ_API vlaq_status vlaq_quantize_weight_int8(const void* W, int64_t N, int64_t K,
+                                      uint32_t flags, int8_t* codes,
+                                      float* s_w, void* stream);
+
+/* Per-token activation quantization with the same optional RMSNorm /
+ * Hadamard prologue as the NVFP4 variant.  codes out [M, K]; s_x out, M
+ * fp32. */
+VLAQ_API vlaq_status vlaq_quantize_act_int8(const void* X, int64_t M, int64_t K,
+                                   const void* gamma, float eps,
+                                   uint32_t flags, int8_t* codes, float* s_x,
+                                   void* stream);
+
+/* Y[m, n] = bf16_rne( fp32( fp32(acc) * fp32(s_x[m] * s_w[n]) ) + residual )
+ * with acc = sum_k x[m, k] w[n, k] exact in s32 on the tensor cores
+ * (tcgen05 kind::i8; |acc| <= K 127^2 < 2^31) and each fp32 step rounded
+ * once, the residual add included: the output has a single correct value,
+ * independent of tiling and split-K (the integer partials are summed
+ * exactly).  Same argument rules as vlaq_linear_nvfp4. */
+VLAQ_API vlaq_status vlaq_linear_int8(const int8_t* xq, const float* s_x,
+                             const int8_t* wq, const float* s_w,
+                             const void* residual, void* Y, int64_t M,
+                             int64_t N, int64_t K, void* workspace,
+                             size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

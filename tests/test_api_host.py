@@ -138,3 +138,31 @@ def test_scales_to_rowmajor_refuses_bad_k(vq):
     with pytest.raises(vq.VlaqError) as ei:
         vq._check(vq._lib.vlaq_scales_to_rowmajor(16, 16, 4, 3420, None))
     assert ei.value.status == 2 and "3420 / 16 = 213.75" in ei.value.message
+
+
+@pytest.mark.parametrize("g", [0.0, -1.0, float("nan"), float("inf"), -0.0])
+def test_static_scale_must_be_finite_and_positive(vq, g):
+    with pytest.raises(vq.VlaqError) as ei:
+        vq.vlaq_quantize_act_nvfp4_static(FAKE, 4, 256, None, None, 1e-6, 0, g, FAKE, FAKE, FAKE)
+    assert ei.value.status == 1 and "g_static" in ei.value.message
+
+
+def test_static_smoothing_flags_need_factors(vq):
+    with pytest.raises(vq.VlaqError) as ei:
+        vq.vlaq_quantize_act_nvfp4_static(FAKE, 4, 256, None, None, 1e-6, vq.F_SMOOTH_MUL, 1.0, FAKE, FAKE, FAKE)
+    assert ei.value.status == 1
+
+
+def test_int8_entry_points_validate_before_the_device(vq):
+    with pytest.raises(vq.VlaqError) as ei:
+        vq.vlaq_quantize_act_int8(FAKE, 4, 3420, None, 1e-6, 0, FAKE, FAKE)
+    assert ei.value.status == 2
+    with pytest.raises(vq.VlaqError) as ei:
+        vq.vlaq_quantize_weight_int8(FAKE, 4, 96, vq.F_HADAMARD64, FAKE, FAKE)
+    assert ei.value.status == 2
+    with pytest.raises(vq.VlaqError) as ei:
+        vq.vlaq_linear_int8(FAKE, FAKE, FAKE, FAKE, None, FAKE, 4, 60, 256)
+    assert ei.value.status == 2
+    vq.vlaq_quantize_act_int8(None, 0, 256, None, 1e-6, 0, None, None)
+    vq.vlaq_linear_int8(None, None, None, None, None, None, 0, 64, 256)
+    assert vq.vlaq_last_error() == ""

@@ -200,3 +200,69 @@ def test_act_nvfp4_smooth_vs_oracle(M, K, tf, mode):
     ref = oracle.quantize_nvfp4_smooth(bits(X), a, bits(gam), 1e-6, flags)
     assert_nvfp4_equal((xq.cpu().numpy(), xs.cpu().numpy(), xg.cpu().numpy()), ref, M, K,
                        f"smooth M={M} K={K} flags={flags}")
+
+
+# Static (calibrated) global scale: g relative to the tensor's largest
+# per-token g -- equal (no saturation), far below (scales and codes
+# saturate), far above (tiny and zero block scales), and absolute extremes
+# that take the exact-division path for 6 g and S.
+STATIC_RATIOS = [1.0, 1e-3, 0.25, 4.0, 1e6]
+STATIC_ABS = [1e-30, 1e-20, 3e19, 1e36]
+
+
+def _static_run(X, M, K, g, gam=None, a=None, flags=0):
+    m = vq()
+    xq, xs, xg = m.alloc_nvfp4(M, K)
+    m.vlaq_quantize_act_nvfp4_static(X.cuda(), M, K, None if gam is None else gam.cuda(),
+                                     None if a is None else to_dev(a), 1e-6, flags, g, xq, xs, xg)
+    torch.cuda.synchronize()
+    m.vlaq_check()
+    return xq.cpu().numpy(), xs.cpu().numpy(), xg.cpu().numpy()
+
+
+@pytest.mark.parametrize("M,K", [(16, 256), (130, 336), (257, 1024), (5, 18944), (3, 48)])
+@pytest.mark.parametrize("ratio", STATIC_RATIOS)
+def test_act_nvfp4_static_vs_oracle(M, K, ratio):
+    X = _inputs(M, K, 91)
+    _, _, gd = oracle.quantize_nvfp4(bits(X))
+    g = float(np.float32(gd.max() * ratio))
+    ref = oracle.quantize_nvfp4_static(bits(X), g)
+    assert_nvfp4_equal(_static_run(X, M, K, g), ref, M, K, f"static {M}x{K} r{ratio}")
+
+
+@pytest.mark.parametrize("g", STATIC_ABS)
+def test_act_nvfp4_static_extreme_scales(g):
+    X = _inputs(37, 1024, 92)
+    ref = oracle.quantize_nvfp4_static(bits(X), g)
+    assert_nvfp4_equal(_static_run(X, 37, 1024, g), ref, 37, 1024, f"static g={g}")
+
+
+@pytest.mark.parametrize("M,K,tf", [(37, 1024, 3), (1024, 3584, 3), (9, 18944, 2), (64, 3584, 1)])
+@pytest.mark.parametrize("mode", [None, 0, 12])
+@pytest.mark.parametrize("ratio", [1.0, 0.05])
+def test_act_nvfp4_static_fused_vs_oracle(M, K, tf, mode, ratio):
+    X = _inputs(M, K, 93)
+    gam = si.norm_gain(K, 93)
+    a = None if mode is None else _awq_like_smoothing(K, 94)
+    flags = tf | (mode or 0)
+    if a is None:
+        _, _, gd = oracle.quantize_nvfp4(bits(X), bits(gam), 1e-6, tf)
+    else:
+        _, _, gd = oracle.quantize_nvfp4_smooth(bits(X), a, bits(gam), 1e-6, flags)
+    g = float(np.float32(np.median(gd) * ratio))
+    ref = oracle.quantize_nvfp4_static(bits(X), g, a, bits(gam), 1e-6, flags)
+    assert_nvfp4_equal(_static_run(X, M, K, g, gam, a, flags), ref, M, K, f"static fused {M}x{K} f{flags}")
+
+
+def test_act_nvfp4_static_edge_values():
+    K = 256
+    rows = [np.zeros(K, np.float32)]
+    r = np.zeros(K, np.float32); r[::2] = -0.0; r[7] = 6.0; rows.append(r)
+    r = np.full(K, 3e38, np.float32); r[5] = -3.3e38; rows.append(r)
+    r = np.full(K, 1e-38, np.float32); r[3] = 3e-38; rows.append(r)
+    rng = np.random.default_rng(95)
+    r = (rng.standard_normal(K) * np.exp2(rng.integers(-30, 30, K))).astype(np.float32); rows.append(r)
+    X = torch.from_numpy(np.stack(rows)).to(torch.bfloat16)
+    for g in (1.0, 1e-3, 2.0 ** -100, 1e30):
+        ref = oracle.quantize_nvfp4_static(bits(X), g)
+        assert_nvfp4_equal(_static_run(X, X.shape[0], K, g), ref, X.shape[0], K, f"static edge g={g}")

@@ -21,8 +21,11 @@ __all__ = [
     "vlaq_last_error", "vlaq_version", "vlaq_check",
     "vlaq_nvfp4_code_pitch", "vlaq_nvfp4_scale_bytes", "vlaq_linear_workspace_bytes",
     "vlaq_quantize_weight_nvfp4", "vlaq_quantize_act_nvfp4", "vlaq_linear_nvfp4",
+    "vlaq_quantize_act_nvfp4_smooth", "vlaq_quantize_act_nvfp4_static", "vlaq_scales_to_rowmajor",
+    "vlaq_selftest_wait_timeout",
     "vlaq_quantize_weight_fp8", "vlaq_quantize_act_fp8", "vlaq_linear_fp8", "vlaq_linear_nvfp4_noalloc",
-    "alloc_nvfp4", "alloc_fp8", "alloc_workspace",
+    "vlaq_quantize_weight_int8", "vlaq_quantize_act_int8", "vlaq_linear_int8",
+    "alloc_nvfp4", "alloc_fp8", "alloc_int8", "alloc_workspace",
 ]
 
 F_RMSNORM = 1
@@ -61,10 +64,14 @@ _SIGS = {
     "vlaq_quantize_weight_fp8": (ctypes.c_int, [_P, _I64, _I64, _U32, _P, _P, _P]),
     "vlaq_quantize_act_fp8": (ctypes.c_int, [_P, _I64, _I64, _P, _F, _U32, _P, _P, _P]),
     "vlaq_linear_fp8": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
+    "vlaq_quantize_weight_int8": (ctypes.c_int, [_P, _I64, _I64, _U32, _P, _P, _P]),
+    "vlaq_quantize_act_int8": (ctypes.c_int, [_P, _I64, _I64, _P, _F, _U32, _P, _P, _P]),
+    "vlaq_linear_int8": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "vlaq_linear_nvfp4_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "vlaq_scales_to_rowmajor": (ctypes.c_int, [_P, _P, _I64, _I64, _P]),
     "vlaq_selftest_wait_timeout": (ctypes.c_int, [_P]),
     "vlaq_quantize_act_nvfp4_smooth": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _F, _U32, _P, _P, _P, _P]),
+    "vlaq_quantize_act_nvfp4_static": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _F, _U32, _F, _P, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -141,6 +148,11 @@ def vlaq_quantize_act_nvfp4_smooth(X, M, K, gamma, smooth, eps, flags, codes, sc
                                                _ptr(scales), _ptr(g_x), _stream(stream)))
 
 
+def vlaq_quantize_act_nvfp4_static(X, M, K, gamma, smooth, eps, flags, g_static, codes, scales, g_x, stream=None):
+    _check(_lib.vlaq_quantize_act_nvfp4_static(_ptr(X), M, K, _ptr(gamma), _ptr(smooth), eps, flags, g_static,
+                                               _ptr(codes), _ptr(scales), _ptr(g_x), _stream(stream)))
+
+
 def vlaq_selftest_wait_timeout(stream=None):
     _check(_lib.vlaq_selftest_wait_timeout(_stream(stream)))
 
@@ -177,6 +189,21 @@ def vlaq_linear_fp8(xq, s_x, wq, s_w, residual, Y, M, N, K, workspace=None, ws_b
                                 _ptr(workspace), ws_bytes, _stream(stream)))
 
 
+# ------------------------------------------------------------------ INT8
+def vlaq_quantize_weight_int8(W, N, K, flags, codes, s_w, stream=None):
+    _check(_lib.vlaq_quantize_weight_int8(_ptr(W), N, K, flags, _ptr(codes), _ptr(s_w), _stream(stream)))
+
+
+def vlaq_quantize_act_int8(X, M, K, gamma, eps, flags, codes, s_x, stream=None):
+    _check(_lib.vlaq_quantize_act_int8(_ptr(X), M, K, _ptr(gamma), eps, flags, _ptr(codes), _ptr(s_x),
+                                       _stream(stream)))
+
+
+def vlaq_linear_int8(xq, s_x, wq, s_w, residual, Y, M, N, K, workspace=None, ws_bytes=0, stream=None):
+    _check(_lib.vlaq_linear_int8(_ptr(xq), _ptr(s_x), _ptr(wq), _ptr(s_w), _ptr(residual), _ptr(Y), M, N, K,
+                                 _ptr(workspace), ws_bytes, _stream(stream)))
+
+
 # ------------------------------------------------------ buffer allocation
 def alloc_nvfp4(rows: int, K: int, device="cuda", per_tensor: bool = False):
     """(codes u8 [rows, pitch], tiled scales u8 [scale_bytes], g f32 [rows or 1])."""
@@ -190,6 +217,12 @@ def alloc_nvfp4(rows: int, K: int, device="cuda", per_tensor: bool = False):
 def alloc_fp8(rows: int, K: int, device="cuda"):
     """(codes u8 [rows, K], scale f32 [rows])."""
     return (torch.empty(max(rows, 1), K, dtype=torch.uint8, device=device),
+            torch.empty(max(rows, 1), dtype=torch.float32, device=device))
+
+
+def alloc_int8(rows: int, K: int, device="cuda"):
+    """(codes int8 [rows, K], scale f32 [rows])."""
+    return (torch.empty(max(rows, 1), K, dtype=torch.int8, device=device),
             torch.empty(max(rows, 1), dtype=torch.float32, device=device))
 
 

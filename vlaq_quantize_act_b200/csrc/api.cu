@@ -3,6 +3,7 @@
 // nothing, touches no output and leaves a message in vlaq_last_error().
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <string>
@@ -185,6 +186,33 @@ vlaq_status vlaq_quantize_act_nvfp4_smooth(const void* X, int64_t M, int64_t K, 
   return ok();
 }
 
+vlaq_status vlaq_quantize_act_nvfp4_static(const void* X, int64_t M, int64_t K, const void* gamma,
+                                           const float* smooth, float eps, uint32_t flags, float g_static,
+                                           uint8_t* codes, uint8_t* scales, float* g_x, void* stream) {
+  const char* fn = "vlaq_quantize_act_nvfp4_static";
+  vlaq_status st;
+  if ((st = check_flags(fn, flags, VLAQ_F_RMSNORM | VLAQ_F_HADAMARD64 | VLAQ_F_SMOOTH_AFTER | VLAQ_F_SMOOTH_MUL)))
+    return st;
+  if ((st = check_k(fn, K, flags, true, vlaq::kMaxQuantK))) return st;
+  if (!(g_static > 0.0f) || !std::isfinite(g_static))
+    return fail(VLAQ_ERR_INVALID_ARG, "%s: g_static = %g must be finite and positive", fn, (double)g_static);
+  if ((flags & (VLAQ_F_SMOOTH_AFTER | VLAQ_F_SMOOTH_MUL)) && smooth == nullptr)
+    return fail(VLAQ_ERR_INVALID_ARG, "%s: smoothing flags without smoothing factors", fn);
+  if (M < 0) return fail(VLAQ_ERR_INVALID_ARG, "%s: M = %lld is negative", fn, (long long)M);
+  if (M > 0x7FFFFFFF) return fail(VLAQ_ERR_SHAPE, "%s: M = %lld is too large", fn, (long long)M);
+  if (M == 0) return ok();
+  VLAQ_NONNULL(fn, X);
+  VLAQ_NONNULL(fn, codes);
+  VLAQ_NONNULL(fn, scales);
+  VLAQ_NONNULL(fn, g_x);
+  if (flags & VLAQ_F_RMSNORM) VLAQ_NONNULL(fn, gamma);
+  if ((st = check_device(fn))) return st;
+  cudaError_t e = vlaq::launch_quant_act_nvfp4_static(X, M, K, gamma, smooth, eps, flags, g_static, codes, scales,
+                                                      g_x, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(fn, e);
+  return ok();
+}
+
 vlaq_status vlaq_quantize_weight_nvfp4(const void* W, int64_t N, int64_t K, uint32_t flags, uint8_t* codes,
                                        uint8_t* scales, float* g_w, void* stream) {
   const char* fn = "vlaq_quantize_weight_nvfp4";
@@ -253,19 +281,57 @@ vlaq_status vlaq_quantize_act_fp8(const void* X, int64_t M, int64_t K, const voi
   return ok();
 }
 
+vlaq_status vlaq_quantize_weight_int8(const void* W, int64_t N, int64_t K, uint32_t flags, int8_t* codes,
+                                      float* s_w, void* stream) {
+  const char* fn = "vlaq_quantize_weight_int8";
+  vlaq_status st;
+  if ((st = check_flags(fn, flags, VLAQ_F_HADAMARD64))) return st;
+  if ((st = check_k(fn, K, flags, false, vlaq::kMaxQuantK))) return st;
+  if (N <= 0 || N > 0x7FFFFFFF) return fail(VLAQ_ERR_SHAPE, "%s: N = %lld out of range", fn, (long long)N);
+  VLAQ_NONNULL(fn, W);
+  VLAQ_NONNULL(fn, codes);
+  VLAQ_NONNULL(fn, s_w);
+  if ((st = check_device(fn))) return st;
+  cudaError_t e = vlaq::launch_quant_int8(W, N, K, nullptr, 0.0f, flags, codes, s_w, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(fn, e);
+  return ok();
+}
+
+vlaq_status vlaq_quantize_act_int8(const void* X, int64_t M, int64_t K, const void* gamma, float eps, uint32_t flags,
+                                   int8_t* codes, float* s_x, void* stream) {
+  const char* fn = "vlaq_quantize_act_int8";
+  vlaq_status st;
+  if ((st = check_flags(fn, flags, VLAQ_F_RMSNORM | VLAQ_F_HADAMARD64))) return st;
+  if ((st = check_k(fn, K, flags, false, vlaq::kMaxQuantK))) return st;
+  if (M < 0) return fail(VLAQ_ERR_INVALID_ARG, "%s: M = %lld is negative", fn, (long long)M);
+  if (M > 0x7FFFFFFF) return fail(VLAQ_ERR_SHAPE, "%s: M = %lld is too large", fn, (long long)M);
+  if (M == 0) return ok();
+  VLAQ_NONNULL(fn, X);
+  VLAQ_NONNULL(fn, codes);
+  VLAQ_NONNULL(fn, s_x);
+  if (flags & VLAQ_F_RMSNORM) VLAQ_NONNULL(fn, gamma);
+  if ((st = check_device(fn))) return st;
+  cudaError_t e = vlaq::launch_quant_int8(X, M, K, gamma, eps, flags, codes, s_x, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(fn, e);
+  return ok();
+}
+
 size_t vlaq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
-  // the FP4 and FP8 plans split identically; report the larger to be safe
+  // the NVFP4 and 8-bit (FP8 / INT8) plans split differently; the larger
   const int sms = vlaq::device_sm_count();
   const size_t a = vlaq::plan_gemm(true, M, N, K, sms).ws_bytes;
   const size_t b = vlaq::plan_gemm(false, M, N, K, sms).ws_bytes;
   return a > b ? a : b;
 }
 
-static vlaq_status linear_common(const char* fn, bool fp4, const uint8_t* xq, const uint8_t* xs, const float* xg,
+enum LinearKind { kLinearNvfp4, kLinearFp8, kLinearInt8 };
+
+static vlaq_status linear_common(const char* fn, LinearKind kind, const uint8_t* xq, const uint8_t* xs, const float* xg,
                                  const uint8_t* wq, const uint8_t* ws, const float* wg, const void* residual, void* Y,
                                  int64_t M, int64_t N, int64_t K, void* workspace, size_t ws_bytes, void* stream) {
   vlaq_status st;
+  const bool fp4 = kind == kLinearNvfp4;
   if ((st = check_k(fn, K, 0, fp4, 0))) return st;
   if (M < 0) return fail(VLAQ_ERR_INVALID_ARG, "%s: M = %lld is negative", fn, (long long)M);
   if (N <= 0 || N % 8 != 0)
@@ -292,8 +358,13 @@ static vlaq_status linear_common(const char* fn, bool fp4, const uint8_t* xq, co
                   ws_bytes, workspace ? "" : ", NULL pointer");
     if (!aligned16(workspace)) return fail(VLAQ_ERR_ALIGN, "%s: workspace is not 16-byte aligned", fn);
   }
-  cudaError_t e = vlaq::launch_linear(fp4, xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, ws_bytes, plan,
-                                      vlaq::kWaitBudgetCycles, static_cast<cudaStream_t>(stream));
+  cudaError_t e =
+      kind == kLinearInt8
+          ? vlaq::launch_linear_int8(reinterpret_cast<const int8_t*>(xq), xg, reinterpret_cast<const int8_t*>(wq), wg,
+                                     residual, Y, M, N, K, workspace, plan, vlaq::kWaitBudgetCycles,
+                                     static_cast<cudaStream_t>(stream))
+          : vlaq::launch_linear(fp4, xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, ws_bytes, plan,
+                                vlaq::kWaitBudgetCycles, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(fn, e);
   return ok();
 }
@@ -301,15 +372,23 @@ static vlaq_status linear_common(const char* fn, bool fp4, const uint8_t* xq, co
 vlaq_status vlaq_linear_nvfp4(const uint8_t* xq, const uint8_t* xs, const float* g_x, const uint8_t* wq,
                               const uint8_t* ws, const float* g_w, const void* residual, void* Y, int64_t M, int64_t N,
                               int64_t K, void* workspace, size_t ws_bytes, void* stream) {
-  return linear_common("vlaq_linear_nvfp4", true, xq, xs, g_x, wq, ws, g_w, residual, Y, M, N, K, workspace,
+  return linear_common("vlaq_linear_nvfp4", kLinearNvfp4, xq, xs, g_x, wq, ws, g_w, residual, Y, M, N, K, workspace,
                        ws_bytes, stream);
 }
 
 vlaq_status vlaq_linear_fp8(const uint8_t* xq, const float* s_x, const uint8_t* wq, const float* s_w,
                             const void* residual, void* Y, int64_t M, int64_t N, int64_t K, void* workspace,
                             size_t ws_bytes, void* stream) {
-  return linear_common("vlaq_linear_fp8", false, xq, nullptr, s_x, wq, nullptr, s_w, residual, Y, M, N, K, workspace,
-                       ws_bytes, stream);
+  return linear_common("vlaq_linear_fp8", kLinearFp8, xq, nullptr, s_x, wq, nullptr, s_w, residual, Y, M, N, K,
+                       workspace, ws_bytes, stream);
+}
+
+vlaq_status vlaq_linear_int8(const int8_t* xq, const float* s_x, const int8_t* wq, const float* s_w,
+                             const void* residual, void* Y, int64_t M, int64_t N, int64_t K, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  return linear_common("vlaq_linear_int8", kLinearInt8, reinterpret_cast<const uint8_t*>(xq), nullptr, s_x,
+                       reinterpret_cast<const uint8_t*>(wq), nullptr, s_w, residual, Y, M, N, K, workspace, ws_bytes,
+                       stream);
 }
 
 vlaq_status vlaq_linear_nvfp4_noalloc(const uint8_t* xq, const uint8_t* xs, const float* g_x, const uint8_t* wq,
@@ -333,7 +412,7 @@ vlaq_status vlaq_linear_nvfp4_noalloc(const uint8_t* xq, const uint8_t* xs, cons
     cudaError_t e = vlaq::noalloc_scratch(&scratch);
     if (e != cudaSuccess) return cuda_fail(fn, e);
   }
-  return linear_common(fn, true, xq, xs, g_x, wq, ws, g_w, residual, Y, M, N, K, scratch,
+  return linear_common(fn, kLinearNvfp4, xq, xs, g_x, wq, ws, g_w, residual, Y, M, N, K, scratch,
                        vlaq::kNoallocScratchBytes, stream);
 }
 

@@ -1,19 +1,23 @@
-// Block-scaled FP4 (NVFP4) and FP8 E4M3 GEMM on the sm_100a tensor cores.
+// Block-scaled FP4 (NVFP4), FP8 E4M3 and INT8 GEMM on the sm_100a tensor cores.
 //
 //   Y[m, n] = bf16_rne( acc[m, n] * scale(m, n) + residual[m, n] )
 //   acc[m, n] = sum_b sx[m, b] sw[n, b] sum_{k in b} e2m1(x[m, k]) e2m1(w[n, k])   (NVFP4)
 //             = sum_k e4m3(x[m, k]) e4m3(w[n, k])                                 (FP8)
-//   scale = g_x[m] * g_w (NVFP4) or s_x[m] * s_w[n] (FP8)
+//             = sum_k x[m, k] w[n, k], exact in s32                               (INT8)
+//   scale = g_x[m] * g_w (NVFP4) or s_x[m] * s_w[n] (FP8, INT8)
+// INT8 rounds each epilogue step once (fp32(acc), s_x s_w, product, residual
+// add), so its output is exact: one value, whatever the split or order.
 //
 // Two persistent, warp-specialised kernels, one CTA per SM, both fed by TMA
 // (2-D tiled loads of the packed codes with 128-byte swizzle) through a ring
-// of shared-memory stages, accumulating 128 x BN fp32 tiles in TMEM with
+// of shared-memory stages, accumulating 128 x BN tiles in TMEM with
 // tcgen05.mma issued from one thread:
 //   gemm_fp4_sfw_kernel  NVFP4, 128 x 256 tiles, kind::mxf4nvf4 with block-16
 //                        UE4M3 scale vectors that four warps write into TMEM;
 //                        split-K (decode shapes) reduced in-kernel by the
 //                        last split of each tile;
-//   gemm_fp8_kernel<BN>  FP8 E4M3, kind::f8f6f4, 128 x 256 or 128 x 128 tiles
+//   gemm_fp8_kernel<BN, I8>  FP8 E4M3 (kind::f8f6f4, fp32 accumulators) or
+//                        INT8 (kind::i8, s32), 128 x 256 or 128 x 128 tiles
 //                        (double-buffered accumulator); split-K partials are
 //                        added by splitk_reduce_kernel in fixed order.
 // Epilogues: tcgen05.ld of the accumulator, scale, residual add, bf16 round,
@@ -40,8 +44,9 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kTmemCols = 512;
 
-// FP8 kernel shape: tile 128 x BN, stages of K = 128 E4M3 elements.
-template <int BN>
+// 8-bit kernel shape: tile 128 x BN, stages of K = 128 E4M3 (or INT8)
+// elements.
+template <int BN, bool I8 = false>
 struct Fp8Cfg {
   static constexpr int A_BYTES = kBM * 128;
   static constexpr int B_BYTES = BN * 128;
@@ -55,8 +60,11 @@ struct Fp8Cfg {
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static_assert(ACC_BUFS * BN <= kTmemCols, "TMEM budget");
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
-  // instruction descriptor: kind::f8f6f4, E4M3 x E4M3, fp32 D, M = 128, N = BN
-  static constexpr uint32_t IDESC = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
+  // instruction descriptor: kind::f8f6f4, E4M3 x E4M3, fp32 D (bits 4-5 =
+  // 1), or kind::i8, signed x signed (bits 7-9, 10-12 = 1), s32 D (bits 4-5
+  // = 2), no saturation; N = BN (bits 17-22, N / 8), M = 128 (bits 24-28, M / 16)
+  static constexpr uint32_t IDESC = (I8 ? (2u << 4) | (1u << 7) | (1u << 10) : (1u << 4)) |
+                                    (uint32_t(BN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
 };
 
 struct GemmArgs {
@@ -118,7 +126,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// fp32 partial sums of one 32-column row segment (split-K).
+// Partial sums of one 32-column row segment (split-K): the accumulator bits
+// as they are (fp32, or s32 for INT8).
 __device__ __forceinline__ void store_partial(const GemmArgs& a, int split, int row, int col0,
                                               const uint32_t (&r)[32]) {
   float* dst = a.partial + (static_cast<size_t>(split) * a.M + row) * a.N + col0;
@@ -129,27 +138,42 @@ __device__ __forceinline__ void store_partial(const GemmArgs& a, int split, int 
     } else {
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        reinterpret_cast<float4*>(dst)[j] =
-            make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                        __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+        reinterpret_cast<uint4*>(dst)[j] = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
     }
   } else {
+    uint32_t* dw = reinterpret_cast<uint32_t*>(dst);
 #pragma unroll
     for (int j = 0; j < 32; ++j)
-      if (col0 + j < a.N) dst[j] = __uint_as_float(r[j]);
+      if (col0 + j < a.N) dw[j] = r[j];
   }
 }
 
+// INT8 epilogue value before the residual: fp32(acc) * fp32(s_x s_w), each
+// step rounded once (no contraction), the order the integer path defines.
+__device__ __forceinline__ float int8_scaled(uint32_t acc_bits, float sx, float sw) {
+  return __fmul_rn(__int2float_rn(static_cast<int>(acc_bits)), __fmul_rn(sx, sw));
+}
+
+// y + residual: one rounding for INT8 (exact output), free otherwise.
+template <bool I8>
+__device__ __forceinline__ float add_residual(float y, float r) {
+  return I8 ? __fadd_rn(y, r) : y + r;
+}
+
 // Scale, residual add, bf16 round and store of one 32-column row segment.
-template <bool FP4>
+template <bool FP4, bool I8 = false>
 __device__ __forceinline__ void store_output(const GemmArgs& a, int row, int col0, float rs,
                                              const uint32_t (&r)[32]) {
   const bool full = col0 + 32 <= a.N;
   float y[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
-    const float sc = FP4 ? rs : rs * ((col0 + j < a.N) ? a.wg[col0 + j] : 0.0f);
-    y[j] = __uint_as_float(r[j]) * sc;
+    if constexpr (FP4) {
+      y[j] = __uint_as_float(r[j]) * rs;  // rs = g_x[m] g_w (one global weight scale)
+    } else {
+      const float sw = (col0 + j < a.N) ? a.wg[col0 + j] : 0.0f;  // per-row weight scale
+      y[j] = I8 ? int8_scaled(r[j], rs, sw) : __uint_as_float(r[j]) * (rs * sw);
+    }
   }
   const size_t base = static_cast<size_t>(row) * a.N + col0;
   if (a.residual) {
@@ -161,14 +185,14 @@ __device__ __forceinline__ void store_output(const GemmArgs& a, int row, int col
         const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          y[8 * j + 2 * t] += __uint_as_float(wv[t] << 16);
-          y[8 * j + 2 * t + 1] += __uint_as_float(wv[t] & 0xFFFF0000u);
+          y[8 * j + 2 * t] = add_residual<I8>(y[8 * j + 2 * t], __uint_as_float(wv[t] << 16));
+          y[8 * j + 2 * t + 1] = add_residual<I8>(y[8 * j + 2 * t + 1], __uint_as_float(wv[t] & 0xFFFF0000u));
         }
       }
     } else {
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        if (col0 + j < a.N) y[j] += __bfloat162float(a.residual[base + j]);
+        if (col0 + j < a.N) y[j] = add_residual<I8>(y[j], __bfloat162float(a.residual[base + j]));
     }
   }
   if (full) {
@@ -192,14 +216,15 @@ __device__ __forceinline__ void store_output(const GemmArgs& a, int row, int col
   }
 }
 
-// FP8 E4M3 W8A8 GEMM: 64 + 32 EPI_WARPS threads, warp 0 TMA producer, warp
-// 1 TMEM allocator and MMA issuer (kind::f8f6f4), the rest epilogue warps;
-// split-K partials are added by splitk_reduce_kernel.
-template <int BN>
-__global__ void __launch_bounds__(Fp8Cfg<BN>::THREADS, 1)
+// 8-bit W8A8 GEMM, FP8 E4M3 (kind::f8f6f4, fp32 accumulators) or INT8
+// (I8: kind::i8, exact s32 accumulators): 64 + 32 EPI_WARPS threads, warp 0
+// TMA producer, warp 1 TMEM allocator and MMA issuer, the rest epilogue
+// warps; split-K partials are added by splitk_reduce_kernel.
+template <int BN, bool I8>
+__global__ void __launch_bounds__(Fp8Cfg<BN, I8>::THREADS, 1)
 gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmArgs args) {
-  using C = Fp8Cfg<BN>;
+  using C = Fp8Cfg<BN, I8>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[C::STAGES];
   __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
@@ -307,9 +332,14 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           uint8_t* sb = sa + C::A_BYTES;
           const int steps = min(4, args.k_steps - 4 * kt);
           const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
-          for (int j = 0; j < steps; ++j)
-            mma_f8f6f4(d_tmem, sdesc_kmajor_sw128(a0 + 32 * j), sdesc_kmajor_sw128(b0 + 32 * j), C::IDESC,
-                       (kt > w.kt0 || j > 0) ? 1u : 0u);
+          for (int j = 0; j < steps; ++j) {
+            const uint64_t ad = sdesc_kmajor_sw128(a0 + 32 * j), bd = sdesc_kmajor_sw128(b0 + 32 * j);
+            const uint32_t accum = (kt > w.kt0 || j > 0) ? 1u : 0u;
+            if constexpr (I8)
+              mma_i8(d_tmem, ad, bd, C::IDESC, accum);
+            else
+              mma_f8f6f4(d_tmem, ad, bd, C::IDESC, accum);
+          }
           umma_commit(&empty_bar[stage]);
           if (++stage == C::STAGES) {
             stage = 0;
@@ -371,7 +401,7 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           if (args.splits > 1)
             store_partial(args, w.split, row, col0, r[c]);
           else
-            store_output<false>(args, row, col0, rs, r[c]);
+            store_output<false, I8>(args, row, col0, rs, r[c]);
         }
       }
     }
@@ -782,8 +812,9 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 }
 
 // Split-K reduction + epilogue: fixed split order, same scaling as the
-// direct epilogue.  8 outputs per thread.
-template <bool FP4>
+// direct epilogue (INT8: exact s32 sums, then the INT8 epilogue steps).
+// 8 outputs per thread.
+template <bool FP4, bool I8 = false>
 __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int splits, int M, int N,
                                      const float* __restrict__ xg, const float* __restrict__ wg,
                                      const __nv_bfloat16* __restrict__ residual,
@@ -796,26 +827,38 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int spli
   const int64_t e0 = idx8 * 8;
   const int row = static_cast<int>(e0 / N);
   const int col = static_cast<int>(e0 % N);
-  float acc[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
-  for (int s = 0; s < splits; ++s) {
-    const float4* p = reinterpret_cast<const float4*>(partial + (static_cast<size_t>(s) * M) * N + e0);
-    const float4 a = p[0], b = p[1];
-    acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-    acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
-  }
-  const float rs = FP4 ? xg[row] * wg[0] : xg[row];
   float y[8];
+  if constexpr (I8) {
+    int acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int s = 0; s < splits; ++s) {
+      const int4* p = reinterpret_cast<const int4*>(partial + (static_cast<size_t>(s) * M) * N + e0);
+      const int4 a = p[0], b = p[1];
+      acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+      acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    }
 #pragma unroll
-  for (int j = 0; j < 8; ++j) y[j] = acc[j] * (FP4 ? rs : rs * wg[col + j]);
+    for (int j = 0; j < 8; ++j) y[j] = int8_scaled(static_cast<uint32_t>(acc[j]), xg[row], wg[col + j]);
+  } else {
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+    for (int s = 0; s < splits; ++s) {
+      const float4* p = reinterpret_cast<const float4*>(partial + (static_cast<size_t>(s) * M) * N + e0);
+      const float4 a = p[0], b = p[1];
+      acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+      acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    }
+    const float rs = FP4 ? xg[row] * wg[0] : xg[row];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = acc[j] * (FP4 ? rs : rs * wg[col + j]);
+  }
   if (residual) {
     const uint4 v = *reinterpret_cast<const uint4*>(residual + e0);
     const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
-      y[2 * t] += __uint_as_float(wv[t] << 16);
-      y[2 * t + 1] += __uint_as_float(wv[t] & 0xFFFF0000u);
+      y[2 * t] = add_residual<I8>(y[2 * t], __uint_as_float(wv[t] << 16));
+      y[2 * t + 1] = add_residual<I8>(y[2 * t + 1], __uint_as_float(wv[t] & 0xFFFF0000u));
     }
   }
   *reinterpret_cast<uint4*>(Y + e0) = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
@@ -903,19 +946,20 @@ cudaError_t run_fp4(const uint8_t* xq, const uint8_t* xs, const float* xg, const
   return launch_pdl(gemm_fp4_sfw_kernel, dim3(grid), dim3(SfwCfg::THREADS), SfwCfg::SMEM_BYTES, s, ta, tb, a);
 }
 
-// FP8: gemm_fp8_kernel<BN>, then the ordered split-K reduction when split.
-template <int BN>
+// FP8 / INT8: gemm_fp8_kernel<BN, I8>, then the ordered split-K reduction
+// when split.
+template <int BN, bool I8>
 cudaError_t run_fp8(const uint8_t* xq, const float* xg, const uint8_t* wq, const float* wg, const void* residual,
                     void* Y, int64_t M, int64_t N, int64_t K, void* workspace, const GemmPlan& plan,
                     long long budget, cudaStream_t s) {
-  using C = Fp8Cfg<BN>;
+  using C = Fp8Cfg<BN, I8>;
   CUtensorMap ta, tb;
   if (!make_map(&ta, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(K), kBM) ||
       !make_map(&tb, wq, static_cast<uint64_t>(K), static_cast<uint64_t>(N), static_cast<uint64_t>(K), BN))
     return cudaErrorInvalidValue;
   const GemmArgs a = make_args(false, BN, nullptr, xg, nullptr, wg, residual, Y, M, N, K, workspace, plan, budget);
   const int grid = plan.grid < a.units ? plan.grid : a.units;
-  auto kern = gemm_fp8_kernel<BN>;
+  auto kern = gemm_fp8_kernel<BN, I8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, s, ta, tb, a);
@@ -923,7 +967,7 @@ cudaError_t run_fp8(const uint8_t* xq, const float* xg, const uint8_t* wq, const
   const int64_t total8 = M * N / 8;
   const int threads = 256;
   const int64_t blocks = (total8 + threads - 1) / threads;
-  return launch_pdl(splitk_reduce_kernel<false>, dim3(static_cast<unsigned int>(blocks)), dim3(threads), 0, s,
+  return launch_pdl(splitk_reduce_kernel<false, I8>, dim3(static_cast<unsigned int>(blocks)), dim3(threads), 0, s,
                     static_cast<const float*>(a.partial), plan.splits, a.M, a.N, xg, wg,
                     static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(Y));
 }
@@ -986,8 +1030,17 @@ cudaError_t launch_linear(bool fp4, const uint8_t* xq, const uint8_t* xs, const 
                           cudaStream_t s) {
   (void)ws_bytes;
   if (fp4) return run_fp4(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
-  if (plan.bn == 256) return run_fp8<256>(xq, xg, wq, wg, residual, Y, M, N, K, workspace, plan, budget, s);
-  return run_fp8<128>(xq, xg, wq, wg, residual, Y, M, N, K, workspace, plan, budget, s);
+  if (plan.bn == 256) return run_fp8<256, false>(xq, xg, wq, wg, residual, Y, M, N, K, workspace, plan, budget, s);
+  return run_fp8<128, false>(xq, xg, wq, wg, residual, Y, M, N, K, workspace, plan, budget, s);
+}
+
+cudaError_t launch_linear_int8(const int8_t* xq, const float* s_x, const int8_t* wq, const float* s_w,
+                               const void* residual, void* Y, int64_t M, int64_t N, int64_t K, void* workspace,
+                               const GemmPlan& plan, long long budget, cudaStream_t s) {
+  const uint8_t* x8 = reinterpret_cast<const uint8_t*>(xq);
+  const uint8_t* w8 = reinterpret_cast<const uint8_t*>(wq);
+  if (plan.bn == 256) return run_fp8<256, true>(x8, s_x, w8, s_w, residual, Y, M, N, K, workspace, plan, budget, s);
+  return run_fp8<128, true>(x8, s_x, w8, s_w, residual, Y, M, N, K, workspace, plan, budget, s);
 }
 
 cudaError_t read_and_clear_status(unsigned int* out, cudaStream_t s) {

@@ -35,10 +35,15 @@ cudaError_t launch_quant_act_nvfp4(const void* X, int64_t M, int64_t K, const vo
 cudaError_t launch_quant_act_nvfp4_smooth(const void* X, int64_t M, int64_t K, const void* gamma,
                                           const float* smooth, float eps, uint32_t flags, uint8_t* codes,
                                           uint8_t* scales, float* g_x, cudaStream_t s);
+cudaError_t launch_quant_act_nvfp4_static(const void* X, int64_t M, int64_t K, const void* gamma, const float* smooth,
+                                          float eps, uint32_t flags, float g_static, uint8_t* codes, uint8_t* scales,
+                                          float* g_x, cudaStream_t s);
 cudaError_t launch_quant_weight_nvfp4(const void* W, int64_t N, int64_t K, uint32_t flags,
                                       uint8_t* codes, uint8_t* scales, float* g_w, cudaStream_t s);
 cudaError_t launch_quant_fp8(const void* X, int64_t rows, int64_t K, const void* gamma, float eps,
                              uint32_t flags, uint8_t* codes, float* s_out, cudaStream_t s);
+cudaError_t launch_quant_int8(const void* X, int64_t rows, int64_t K, const void* gamma, float eps,
+                              uint32_t flags, int8_t* codes, float* s_out, cudaStream_t s);
 cudaError_t launch_scales_to_rowmajor(const uint8_t* in, uint8_t* out, int64_t rows, int64_t K, cudaStream_t s);
 
 // ---- GEMM (gemm.cu)
@@ -59,6 +64,9 @@ inline size_t splitk_partial_bytes(int64_t splits, int64_t M, int64_t N) {
   return (static_cast<size_t>(splits) * M * N * sizeof(float) + 255) / 256 * 256;
 }
 
+cudaError_t launch_linear_int8(const int8_t* xq, const float* s_x, const int8_t* wq, const float* s_w,
+                               const void* residual, void* Y, int64_t M, int64_t N, int64_t K, void* workspace,
+                               const GemmPlan& plan, long long budget, cudaStream_t s);
 cudaError_t launch_linear(bool fp4, const uint8_t* xq, const uint8_t* xs, const float* xg,
                           const uint8_t* wq, const uint8_t* ws, const float* wg,
                           const void* residual, void* Y, int64_t M, int64_t N, int64_t K,

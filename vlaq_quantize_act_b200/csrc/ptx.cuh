@@ -144,6 +144,18 @@ __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t adesc, uint
       : "memory");
 }
 
+// D(tmem) (+)= A(smem) * B(smem)^T, signed INT8 x INT8, s32 accumulate
+// (exact: no saturation bit in the descriptor, |sums| < 2^31 here).
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // 32 lanes x 4 consecutive 32-bit columns from registers: thread i writes
 // lane (base + i).  Completion is awaited with tmem_st_wait().
 __device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint4& v) {

@@ -41,8 +41,8 @@ __device__ unsigned int g_vlaq_quant_status = 0;
 
 namespace {
 
-enum { kNvfp4 = 0, kFp8 = 1 };
-enum { kPerRow = 0, kTensorAmax = 1, kTensorQuant = 2 };
+enum { kNvfp4 = 0, kFp8 = 1, kInt8 = 2 };
+enum { kPerRow = 0, kTensorAmax = 1, kTensorQuant = 2, kStatic = 3 };
 
 constexpr int kMaxRowBufs = 4;
 constexpr int kShortRowK = 8192;  // rows up to this length take the 8-warp CTAs
@@ -147,6 +147,7 @@ struct RowArgs {
   int64_t rows;
   const float* smooth;  // per-input-channel smoothing factors [K] (or null)
   uint32_t sflags;      // kFlagSmoothAfter | kFlagSmoothMul
+  float g_static;       // calibrated global scale (kStatic)
   int nbuf;       // ring depth (rows in flight per CTA)
   int row_bytes;  // ring slot size (2 K rounded up to 128)
   long long budget;
@@ -229,8 +230,8 @@ __device__ __forceinline__ float absmax16(const float* v) {
 }
 
 // All rows of one launch: FMT (NVFP4 / FP8), MODE (per-row scale, tensor
-// amax pass, tensor quantize pass), NORM (RMSNorm, per-row modes only), WHT
-// (block-64 Hadamard), W warps per CTA.  Persistent grid: the CTA takes rows
+// amax pass, tensor quantize pass, static calibrated scale), NORM (RMSNorm,
+// per-row and static modes), WHT (block-64 Hadamard), W warps per CTA.  Persistent grid: the CTA takes rows
 // blockIdx.x + i gridDim.x, the ring slot of row i is i mod nbuf.
 template <int FMT, int MODE, bool NORM, bool WHT, bool SMOOTH, int W>
 __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) quant_rows_kernel(const RowArgs a) {
@@ -269,6 +270,7 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
   }
   float g_tensor = 0.0f;
   if (MODE == kTensorQuant) g_tensor = __fdiv_rn(__uint_as_float(*a.amax_word), 2688.0f);
+  if (MODE == kStatic) g_tensor = a.g_static;
 
   int slot = 0;
   uint32_t phase = 0;
@@ -319,7 +321,8 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
     // ---- pass A: per-block amax (kept in registers) and row amax
     float a16r[MAXIT];
     float g = g_tensor;
-    if (MODE != kTensorQuant) {
+    if (MODE == kStatic && tid == 0) a.gout[row] = g;
+    if (MODE == kPerRow || MODE == kTensorAmax) {
       float local = 0.0f;
 #pragma unroll
       for (int it = 0; it < MAXIT; ++it) {
@@ -349,7 +352,7 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
       if (MODE == kTensorAmax) {
         if (tid == 0) atomicMax(a.amax_word, __float_as_uint(A));  // A >= 0: bit order = value order
       } else {
-        g = (FMT == kNvfp4) ? __fdiv_rn(A, 2688.0f) : __fdiv_rn(A, 448.0f);
+        g = (FMT == kNvfp4) ? __fdiv_rn(A, 2688.0f) : __fdiv_rn(A, FMT == kFp8 ? 448.0f : 127.0f);
         if (tid == 0) a.gout[row] = g;
       }
     }
@@ -366,14 +369,24 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
             const int q = (it * W + warp) * 32 + lane;
             float v[16];
             block_values<NORM, WHT, SMOOTH>(a, rs, q, nblk16, r, lane, v);
-            const float a16 = (MODE == kPerRow) ? a16r[it] : absmax16(v);
+            float a16 = (MODE == kPerRow) ? a16r[it] : absmax16(v);
             uint32_t sb8 = 0;
             float S = 0.0f;
             if (g > 0.0f) {
+              // A calibrated g bounds neither a16 / 6 g nor v / S: values
+              // whose quotient would pass 512 (scale 448 either way) or 8
+              // (code 6 either way) are clamped there (exact: powers of two),
+              // so no quotient overflows, in the correction step or a divide.
+              if (MODE == kStatic) a16 = fminf(a16, __fmul_rn(512.0f, d6g.S));
               sb8 = e4m3_of_quotient(a16, d6g);
               S = __fmul_rn(e4m3_to_f32(sb8), g);
             }
             const Divisor dv = make_divisor(S);
+            if (MODE == kStatic) {
+              const float b = __fmul_rn(8.0f, S);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) v[j] = fminf(fmaxf(v[j], -b), b);
+            }
             float qv[16];
             quotients<16>(v, dv, qv);
             const uint32_t w0 = cvt_e2m1x8(qv);
@@ -395,9 +408,23 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
             float qv[16];
             quotients<16>(v, dg, qv);
             uint32_t w[4];
+            if (FMT == kInt8) {
+              // round half to even, clamp to [-127, 127], two's complement bytes
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              w[j] = cvt_e4m3x2(qv[4 * j], qv[4 * j + 1]) | (cvt_e4m3x2(qv[4 * j + 2], qv[4 * j + 3]) << 16);
+              for (int j = 0; j < 4; ++j) {
+                uint32_t word = 0;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                  const int c = min(127, max(-127, __float2int_rn(qv[4 * j + t])));
+                  word |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * t);
+                }
+                w[j] = word;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                w[j] = cvt_e4m3x2(qv[4 * j], qv[4 * j + 1]) | (cvt_e4m3x2(qv[4 * j + 2], qv[4 * j + 3]) << 16);
+            }
             if (q < nblk16) *reinterpret_cast<uint4*>(crow + 16 * q) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
@@ -456,7 +483,7 @@ cudaError_t launch_shape(const RowArgs& a, cudaStream_t s) {
 template <int FMT, int MODE>
 cudaError_t launch_rows(const void* X, int64_t rows, int64_t K, const void* gamma, float eps, uint32_t flags,
                         uint8_t* codes, int64_t pitch, uint8_t* scales, float* gout, unsigned int* amax,
-                        cudaStream_t s, const float* smooth = nullptr) {
+                        cudaStream_t s, const float* smooth = nullptr, float g_static = 0.0f) {
   RowArgs a;
   a.X = static_cast<const __nv_bfloat16*>(X);
   a.K = static_cast<int>(K);
@@ -470,18 +497,19 @@ cudaError_t launch_rows(const void* X, int64_t rows, int64_t K, const void* gamm
   a.rows = rows;
   a.smooth = smooth;
   a.sflags = flags & (kFlagSmoothAfter | kFlagSmoothMul);
+  a.g_static = g_static;
   a.nbuf = 0;
   a.row_bytes = static_cast<int>((2 * K + 127) / 128 * 128);
   a.budget = kWaitBudgetCycles;
   const bool wht = (flags & kFlagHadamard) != 0;
-  if constexpr (MODE == kPerRow && FMT == kNvfp4) {
+  if constexpr ((MODE == kPerRow || MODE == kStatic) && FMT == kNvfp4) {
     if (smooth) {
       if (flags & kFlagRmsNorm)
         return wht ? launch_shape<FMT, MODE, true, true, true>(a, s) : launch_shape<FMT, MODE, true, false, true>(a, s);
       return wht ? launch_shape<FMT, MODE, false, true, true>(a, s) : launch_shape<FMT, MODE, false, false, true>(a, s);
     }
   }
-  if constexpr (MODE == kPerRow) {
+  if constexpr (MODE == kPerRow || MODE == kStatic) {
     if (flags & kFlagRmsNorm)
       return wht ? launch_shape<FMT, MODE, true, true>(a, s) : launch_shape<FMT, MODE, true, false>(a, s);
   }
@@ -503,6 +531,13 @@ cudaError_t launch_quant_act_nvfp4_smooth(const void* X, int64_t M, int64_t K, c
                                       s, smooth);
 }
 
+cudaError_t launch_quant_act_nvfp4_static(const void* X, int64_t M, int64_t K, const void* gamma, const float* smooth,
+                                          float eps, uint32_t flags, float g_static, uint8_t* codes, uint8_t* scales,
+                                          float* g_x, cudaStream_t s) {
+  return launch_rows<kNvfp4, kStatic>(X, M, K, gamma, eps, flags, codes, nvfp4_code_pitch(K), scales, g_x, nullptr,
+                                      s, smooth, g_static);
+}
+
 cudaError_t launch_quant_weight_nvfp4(const void* W, int64_t N, int64_t K, uint32_t flags, uint8_t* codes,
                                       uint8_t* scales, float* g_w, cudaStream_t s) {
   // Three steps, no scratch memory: the tensor amax is accumulated in g_w
@@ -522,6 +557,12 @@ cudaError_t launch_quant_weight_nvfp4(const void* W, int64_t N, int64_t K, uint3
 cudaError_t launch_quant_fp8(const void* X, int64_t rows, int64_t K, const void* gamma, float eps, uint32_t flags,
                              uint8_t* codes, float* s_out, cudaStream_t s) {
   return launch_rows<kFp8, kPerRow>(X, rows, K, gamma, eps, flags, codes, K, nullptr, s_out, nullptr, s);
+}
+
+cudaError_t launch_quant_int8(const void* X, int64_t rows, int64_t K, const void* gamma, float eps, uint32_t flags,
+                              int8_t* codes, float* s_out, cudaStream_t s) {
+  return launch_rows<kInt8, kPerRow>(X, rows, K, gamma, eps, flags, reinterpret_cast<uint8_t*>(codes), K, nullptr,
+                                     s_out, nullptr, s);
 }
 
 namespace {
