@@ -236,7 +236,7 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
 // nibble of the low byte.
 __device__ __forceinline__ uint32_t cvt_e2m1x8(const float* v) {
   uint32_t out;
-  asm volatile(
+  asm(
       "{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
@@ -251,7 +251,7 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float* v) {
 // Two fp32 -> two E4M3 bytes (RNE, saturating), `lo` in the low byte.
 __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   uint16_t out;
-  asm volatile("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(hi), "f"(lo));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(hi), "f"(lo));
   return out;
 }
 
@@ -259,7 +259,7 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
 __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
   uint32_t h2;
   const uint16_t in = static_cast<uint16_t>(byte & 0xFFu);
-  asm volatile("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
   return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
 }
 

@@ -45,6 +45,7 @@ enum { kNvfp4 = 0, kFp8 = 1, kInt8 = 2 };
 enum { kPerRow = 0, kTensorAmax = 1, kTensorQuant = 2, kStatic = 3 };
 
 constexpr int kMaxRowBufs = 4;
+constexpr int kMidRowK = 4096;    // many rows up to this length: 4-warp CTAs, 8 per SM
 constexpr int kShortRowK = 8192;  // rows up to this length take the 8-warp CTAs
 
 // CTA shape per row length: W warps, CTAs resident per SM, ring budget.
@@ -52,7 +53,8 @@ template <int W>
 struct RowCfg {
   static constexpr int kThreads = 32 * W;
   static constexpr int kCtasPerSm = 1024 / kThreads;  // 32 warps per SM, 64 registers a thread
-  static constexpr int kRingBytes = (W == 8) ? 52 * 1024 : 110 * 1024;
+  static constexpr int kRingBytes = (W == 4) ? 26 * 1024 : (W == 8) ? 52 * 1024 : 110 * 1024;
+  static constexpr int kMaxK = (W == 4) ? kMidRowK : (W == 8) ? kShortRowK : int(kMaxQuantK);
 };
 
 __device__ __forceinline__ void unpack_bf16x8(const uint4& q, float* v) {
@@ -236,7 +238,7 @@ __device__ __forceinline__ float absmax16(const float* v) {
 template <int FMT, int MODE, bool NORM, bool WHT, bool SMOOTH, int W>
 __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) quant_rows_kernel(const RowArgs a) {
   constexpr int T = RowCfg<W>::kThreads;
-  constexpr int MAXIT = (W == 8 ? kShortRowK : int(kMaxQuantK)) / 16 / T;  // blocks per lane, at most
+  constexpr int MAXIT = RowCfg<W>::kMaxK / 16 / T;  // blocks per lane, at most
   extern __shared__ __align__(128) uint8_t s_ring[];
   __shared__ __align__(8) uint64_t s_bar[kMaxRowBufs];
   __shared__ float s_red[W];
@@ -327,7 +329,7 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
 #pragma unroll
       for (int it = 0; it < MAXIT; ++it) {
         a16r[it] = 0.0f;
-        if (it < iters) {
+        if (it < iters && (it * W + warp) * 32 < nblk16_pad) {
           const int q = (it * W + warp) * 32 + lane;
           float m = 0.0f;
           if (NORM || WHT || SMOOTH) {
@@ -342,8 +344,8 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
           local = fmaxf(local, m);
         }
       }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) local = fmaxf(local, __shfl_xor_sync(0xffffffffu, local, o));
+      // non-negative floats order like their bit patterns: one warp reduction
+      local = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(local)));
       if (lane == 0) s_red[warp] = local;
       __syncthreads();
       float A = s_red[0];
@@ -365,7 +367,7 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
         const Divisor d6g = make_divisor(__fmul_rn(6.0f, g));
 #pragma unroll
         for (int it = 0; it < MAXIT; ++it) {
-          if (it < iters) {
+          if (it < iters && (it * W + warp) * 32 < nblk16_pad) {
             const int q = (it * W + warp) * 32 + lane;
             float v[16];
             block_values<NORM, WHT, SMOOTH>(a, rs, q, nblk16, r, lane, v);
@@ -401,7 +403,7 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
         const Divisor dg = make_divisor(g);
 #pragma unroll
         for (int it = 0; it < MAXIT; ++it) {
-          if (it < iters) {
+          if (it < iters && (it * W + warp) * 32 < nblk16_pad) {
             const int q = (it * W + warp) * 32 + lane;
             float v[16];
             block_values<NORM, WHT, SMOOTH>(a, rs, q, nblk16, r, lane, v);
@@ -476,6 +478,10 @@ cudaError_t launch_ring(RowArgs a, cudaStream_t s) {
 
 template <int FMT, int MODE, bool NORM, bool WHT, bool SMOOTH = false>
 cudaError_t launch_shape(const RowArgs& a, cudaStream_t s) {
+  // short rows and enough of them for every SM: one row per small CTA, so
+  // more rows are worked on at once; few rows keep the 8-warp CTAs (shorter
+  // per-row chains)
+  if (a.K <= kMidRowK && a.rows >= 2 * device_sm_count()) return launch_ring<FMT, MODE, NORM, WHT, SMOOTH, 4>(a, s);
   if (a.K <= kShortRowK) return launch_ring<FMT, MODE, NORM, WHT, SMOOTH, 8>(a, s);
   return launch_ring<FMT, MODE, NORM, WHT, SMOOTH, 16>(a, s);
 }
