@@ -124,7 +124,7 @@ def test_end_to_end_nvfp4(M, N, K, flags, res):
 
 def test_workspace_is_checked():
     m = vq()
-    M, N, K = 1, 512, 4096
+    M, N, K = 8, 512, 4096
     need = m.vlaq_linear_workspace_bytes(M, N, K)
     assert need > 0  # this decode shape runs split-K
     xq, xs, xg = m.alloc_nvfp4(M, K)
@@ -174,7 +174,7 @@ def test_split_workspace_reused_across_calls_and_shapes():
     counts.  A counter left non-zero would keep the next call's last split
     from recognising itself, and its tile would stay NaN."""
     m = vq()
-    shapes = [(1, 512, 4096), (4, 1024, 3584), (8, 256, 2048)]
+    shapes = [(5, 512, 4096), (8, 1024, 3584), (6, 256, 2048)]
     need = max(m.vlaq_linear_workspace_bytes(*s) for s in shapes)
     assert all(m.vlaq_linear_workspace_bytes(*s) > 0 for s in shapes)  # all three split K
     wsp = torch.zeros(need, dtype=torch.uint8, device="cuda")
@@ -197,3 +197,38 @@ def test_split_workspace_reused_across_calls_and_shapes():
                 first[(M, N, K)] = y
             else:
                 assert np.array_equal(y, first[(M, N, K)]), (rep, M, N, K)
+
+
+# one or two token rows against weights of at most 2^25 elements take the
+# weight-streaming CUDA-core kernel (larger M or weights the tensor-core one):
+# ragged K (K % 64 in {16, 32, 48}, K = 16), N = 8, a partial last group of
+# rows per CTA, the decode projection shapes, residual on and off
+FEW_ROW_CASES = [(1, 8, 16, False), (2, 24, 48, True), (3, 136, 208, False), (4, 512, 4096, True),
+                 (1, 4608, 3584, True), (4, 4608, 3584, False), (1, 3584, 18944, True), (2, 3584, 18944, False),
+                 (3, 40, 336, True), (1, 37888, 3584, False)]
+
+
+@pytest.mark.parametrize("M,N,K,res", FEW_ROW_CASES + [(2, 4608, 3584, True), (2, 3584, 3584, False)])
+def test_linear_nvfp4_few_rows(M, N, K, res):
+    m = vq()
+    X = si.projection_activations(K, M, 61)
+    W = si.projection_weight(K, N, 61)
+    cx, sx, gx = oracle.quantize_nvfp4(bits(X))
+    cw, sw, gw = oracle.quantize_nvfp4(bits(W), per_tensor=True)
+    R = si.residual(M, N, 61) if res else None
+    Y64 = oracle.linear_f64(oracle.decode_nvfp4(cx, sx, gx, K), oracle.decode_nvfp4(cw, sw, gw, K, per_tensor=True),
+                            None if R is None else bits(R))
+    dev = (to_dev(layouts.pad_codes(cx, K)), to_dev(layouts.tile_scales(sx, M, K)), to_dev(gx),
+           to_dev(layouts.pad_codes(cw, K)), to_dev(layouts.tile_scales(sw, N, K)), to_dev(gw))
+    Y = gpu_linear_nvfp4(*dev, M, N, K, None if R is None else R.cuda())
+    rel, mx = gemm_error(Y, Y64)
+    print(f"few rows M={M} N={N} K={K}: rel_fro={rel:.3e} max_abs={mx:.3e}")
+    assert rel < REL_FRO_TOL, (rel, mx)
+    # the CUDA-core kernel needs no workspace; a second call gives the same bits
+    few = M <= 2 and N * K <= 1 << 25
+    Y2 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    wsp, nb = (None, 0) if few else m.alloc_workspace(M, N, K)
+    m.vlaq_linear_nvfp4(*dev, None if R is None else R.cuda(), Y2, M, N, K, wsp, nb)
+    torch.cuda.synchronize()
+    m.vlaq_check()
+    assert np.array_equal(Y2.float().cpu().numpy(), Y)

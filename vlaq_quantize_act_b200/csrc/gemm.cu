@@ -979,8 +979,16 @@ GemmPlan plan_gemm(bool fp4, int64_t M, int64_t N, int64_t K, int num_sms) {
   const int64_t k_steps = fp4 ? (K + 63) / 64 : (K + 31) / 32;
   const int64_t k_tiles = (k_steps + 3) / 4;
   const int64_t m_tiles = (M + kBM - 1) / kBM;
+  if (fp4 && gemv_supported(M, N, K)) {
+    // one or two token rows, small weights: the weight-streaming kernel on the CUDA cores
+    p.bn = 0;
+    p.splits = 1;
+    p.grid = 0;
+    p.ws_bytes = 0;
+    return p;
+  }
   if (fp4) {
-    // NVFP4: always the 128 x 256 scale-writer kernel; few output tiles
+    // NVFP4: the 128 x 256 scale-writer kernel; few output tiles
     // (decode) are split along K so every SM streams weights, and the last
     // split of each tile reduces in-kernel (per-tile counters after the
     // partials, zero between calls).
@@ -1029,6 +1037,7 @@ cudaError_t launch_linear(bool fp4, const uint8_t* xq, const uint8_t* xs, const 
                           int64_t K, void* workspace, size_t ws_bytes, const GemmPlan& plan, long long budget,
                           cudaStream_t s) {
   (void)ws_bytes;
+  if (fp4 && plan.bn == 0) return launch_gemv_nvfp4(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, s);
   if (fp4) return run_fp4(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
   if (plan.bn == 256) return run_fp8<256, false>(xq, xg, wq, wg, residual, Y, M, N, K, workspace, plan, budget, s);
   return run_fp8<128, false>(xq, xg, wq, wg, residual, Y, M, N, K, workspace, plan, budget, s);

@@ -48,7 +48,7 @@ cudaError_t launch_scales_to_rowmajor(const uint8_t* in, uint8_t* out, int64_t r
 
 // ---- GEMM (gemm.cu)
 struct GemmPlan {
-  int bn;          // tile width along N
+  int bn;          // tile width along N (0: the few-row CUDA-core kernel)
   int splits;      // split-K factor (1 = direct epilogue)
   int grid;        // persistent CTAs
   size_t ws_bytes; // fp32 partials needed when splits > 1
@@ -67,6 +67,17 @@ inline size_t splitk_partial_bytes(int64_t splits, int64_t M, int64_t N) {
 cudaError_t launch_linear_int8(const int8_t* xq, const float* s_x, const int8_t* wq, const float* s_w,
                                const void* residual, void* Y, int64_t M, int64_t N, int64_t K, void* workspace,
                                const GemmPlan& plan, long long budget, cudaStream_t s);
+// Few-row NVFP4 linear on the CUDA cores (gemv.cu): M <= kGemvMaxM, at most
+// kGemvMaxWeights weight elements, and the expanded activation rows fit two
+// CTAs per SM.
+constexpr int kGemvMaxM = 2;
+constexpr int64_t kGemvMaxWeights = int64_t(1) << 25;
+constexpr size_t kGemvSmemBudget = 200 * 1024;
+size_t gemv_smem_bytes(int64_t M, int64_t K);
+bool gemv_supported(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_gemv_nvfp4(const uint8_t* xq, const uint8_t* xs, const float* xg, const uint8_t* wq,
+                              const uint8_t* ws, const float* wg, const void* residual, void* Y, int64_t M, int64_t N,
+                              int64_t K, cudaStream_t s);
 cudaError_t launch_linear(bool fp4, const uint8_t* xq, const uint8_t* xs, const float* xg,
                           const uint8_t* wq, const uint8_t* ws, const float* wg,
                           const void* residual, void* Y, int64_t M, int64_t N, int64_t K,

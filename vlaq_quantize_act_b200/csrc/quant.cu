@@ -114,8 +114,9 @@ __device__ __forceinline__ float markstein_quotient(float x, float S, float y) {
 // RN(v[i] / S) for N values (0 when S = 0).  Executed by the whole warp.
 template <int N>
 __device__ __forceinline__ void quotients(const float* v, const Divisor& d, float* q) {
+  static_assert(N % 2 == 0, "pairs");
 #pragma unroll
-  for (int i = 0; i < N; ++i) q[i] = markstein_quotient(v[i], d.S, d.y);
+  for (int i = 0; i < N; i += 2) markstein_pair(v[i], v[i + 1], d.S, d.y, q[i], q[i + 1]);
   if (__any_sync(0xffffffffu, d.slow)) {
     if (d.slow) {
 #pragma unroll
