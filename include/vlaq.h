@@ -224,7 +224,10 @@ VLAQ_API size_t vlaq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 /* Y = bf16_rne( (sum_k dec(x)[m,k] * dec(w)[n,k]) + residual[m,n] )
  * with the product accumulated in fp32 on the tensor cores
  * (tcgen05 kind::mxf4nvf4, block-16 E4M3 scales) and the global scales
- * g_x[m] * g_w applied in the epilogue.
+ * g_x[m] * g_w applied in the epilogue.  One or two token rows against a
+ * weight of at most 2^25 elements run on the CUDA cores instead (weight
+ * streaming; each 16-block dot product an exact integer, the block scaling
+ * and the sum over blocks in fp32); those shapes need no workspace.
  *   xq, xs, g_x  activation codes / tiled scales / globals (M rows)
  *   wq, ws, g_w  weight codes / tiled scales / global (N rows)
  *   residual     bf16 [M, N] or NULL
