@@ -205,7 +205,8 @@ def test_split_workspace_reused_across_calls_and_shapes():
 # rows per CTA, the decode projection shapes, residual on and off
 FEW_ROW_CASES = [(1, 8, 16, False), (2, 24, 48, True), (3, 136, 208, False), (4, 512, 4096, True),
                  (1, 4608, 3584, True), (4, 4608, 3584, False), (1, 3584, 18944, True), (2, 3584, 18944, False),
-                 (3, 40, 336, True), (1, 37888, 3584, False)]
+                 (3, 40, 336, True), (1, 37888, 3584, False),
+                 (2, 1024, 18944, True)]  # the few-row kernel with more than 48 KB of shared memory
 
 
 @pytest.mark.parametrize("M,N,K,res", FEW_ROW_CASES + [(2, 4608, 3584, True), (2, 3584, 3584, False)])

@@ -220,7 +220,7 @@ def _static_run(X, M, K, g, gam=None, a=None, flags=0):
     return xq.cpu().numpy(), xs.cpu().numpy(), xg.cpu().numpy()
 
 
-@pytest.mark.parametrize("M,K", [(16, 256), (130, 336), (257, 1024), (5, 18944), (3, 48)])
+@pytest.mark.parametrize("M,K", [(16, 256), (130, 336), (257, 1024), (5, 18944), (3, 48), (1024, 1024)])
 @pytest.mark.parametrize("ratio", STATIC_RATIOS)
 def test_act_nvfp4_static_vs_oracle(M, K, ratio):
     X = _inputs(M, K, 91)
