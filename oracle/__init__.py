@@ -1,4 +1,4 @@
-"""CPU oracle for the NVFP4 / FP8 quantize + linear path.
+"""CPU oracle for the NVFP4 / FP8 / INT8 quantize + linear path.
 
 TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check and by the
 benchmark's cpu_baseline / reference leg, never by the product package.  It
@@ -8,7 +8,7 @@ exchanges numpy arrays in the *logical* layouts:
 * bf16 inputs as ``uint16`` arrays holding the bf16 bit patterns,
 * NVFP4 codes ``uint8 [rows, K/2]`` (element k in byte k/2, low nibble first),
 * NVFP4 block scales ``uint8 [rows, K/16]`` (E4M3 bytes, row-major),
-* FP8 codes ``uint8 [rows, K]``.
+* FP8 codes ``uint8 [rows, K]``, INT8 codes ``int8 [rows, K]``.
 
 Every function cites the passage it follows in the C source's header.
 """

@@ -1,6 +1,6 @@
 /*
  * vlaq oracle: a plain, slow, obviously correct CPU statement of what the
- * NVFP4 / FP8 quantize + linear path computes.
+ * NVFP4 / FP8 / INT8 quantize + linear path computes.
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, loads or
  * calls this file.  It shares no code, header, table or constant generator
@@ -29,6 +29,14 @@
  *  - FP8 E4M3 W8A8 with per-row weight scale and per-token activation
  *    scale (the FP8 recipe commit of PR #2 uses per-tensor scales; the
  *    per-row / per-token granularity is the stated workload's choice).
+ *  - "FoldQuant W8A8/W4A4 inference ...", the INT8 path: INT8 codes with
+ *    per-row weight scales, activations quantized per token, integer GEMMs
+ *    whose sums are exact in any order (SYCL commit).
+ *  - same page, dequant commit: per-input-channel smoothing x' = R(x / a)
+ *    or R(x) / a; "NVIDIA/TensorRT-Edge-LLM PR #193", pre_quant_scale
+ *    commit: the AWQ pre_quant_scale multiplies the activations, and an
+ *    NVFP4 linear carries input_scale (a static activation global scale)
+ *    beside weight_scale and weight_scale_2.
  *
  * Floating point: quantization runs in IEEE fp32 with every operation
  * rounded once (build with -ffp-contract=off, no -ffast-math); the GEMM
