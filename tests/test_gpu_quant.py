@@ -46,6 +46,25 @@ def test_act_nvfp4_rmsnorm_ragged_k():
     assert_nvfp4_equal(gpu_quant_act_nvfp4(X, gam, 1e-5, 1), ref, 33, 336, "rmsnorm K=336")
 
 
+@pytest.mark.parametrize("M", [1, 300])
+def test_act_nvfp4_rmsnorm_tree_golden_row(M):
+    """The hand-worked row of tests/golden/sumsq_tree.txt through the fused
+    RMSNorm prologue: its global scale separates the page's reduction tree
+    (FoldQuant SYCL commit) from every other summation order, so the kernel's
+    tree is pinned by a value worked by hand, not only by the oracle.  M = 300
+    takes the many-rows CTA shape, M = 1 the few-rows one."""
+    from test_oracle_pins import sumsq_golden
+    x, _, rec = sumsq_golden()
+    K = x.size
+    X = torch.from_numpy(np.tile(x, (M, 1))).to(torch.bfloat16)
+    gam = torch.ones(K, dtype=torch.bfloat16)
+    gam[0] = torch.from_numpy(np.array([int(rec["gain0"], 16)], np.uint16).view(np.int16)).view(torch.bfloat16)[0]
+    got = gpu_quant_act_nvfp4(X, gam, 1e-6, 1)
+    assert (got[2].view(np.uint32)[:M] == int(rec["g_bits"], 16)).all(), [hex(v) for v in got[2].view(np.uint32)[:4]]
+    ref = oracle.quantize_nvfp4(bits(X), bits(gam), 1e-6, 1)
+    assert_nvfp4_equal(got, ref, M, K, "golden tree row")
+
+
 def test_act_nvfp4_tiny_config_outliers():
     X, _ = si.tiny_inputs(0)
     ref = oracle.quantize_nvfp4(bits(X))

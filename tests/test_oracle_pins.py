@@ -317,6 +317,117 @@ def test_sumsq_tree_order_exact_on_small_integers():
     assert float(oracle.sumsq_tree(x)) == float(np.sum(x.astype(np.float64) ** 2))
 
 
+def sumsq_golden():
+    """The hand-worked rows of tests/golden/sumsq_tree.txt."""
+    rec = {"x": {}, "fma_x": {}}
+    for r in _golden_lines("sumsq_tree.txt"):
+        if r[0] in rec:
+            rec[r[0]][int(r[1])] = float(r[2])
+        else:
+            rec[r[0]] = r[1]
+    x = np.zeros(512, np.float32)
+    for k, v in rec["x"].items():
+        x[k] = v
+    xf = np.zeros(8, np.float32)
+    for k, v in rec["fma_x"].items():
+        xf[k] = v
+    return x, xf, rec
+
+
+# Other summation orders of the same squares (fp32, one rounding per step;
+# a square plus a sum is exact in fp64 for these inputs, so fp64 then one
+# fp32 rounding is the fused multiply-add).
+def _fma(x, acc):
+    return np.float32(np.float64(x) * np.float64(x) + np.float64(acc))
+
+
+def _add(a, b):
+    return np.float32(np.float64(a) + np.float64(b))
+
+
+def _lanes(x, chunk, owner):
+    p = [np.float32(0)] * 32
+    for c in range(len(x) // chunk):
+        lane = owner(c)
+        for e in range(chunk):
+            p[lane] = _fma(x[chunk * c + e], p[lane])
+    return p
+
+
+def _butterfly(p, offsets=(16, 8, 4, 2, 1)):
+    for o in offsets:
+        p = [_add(p[l], p[l ^ o]) for l in range(32)]
+    return p[0]
+
+
+def _pairwise(x):
+    if len(x) == 1:
+        return np.float32(np.float64(x[0]) ** 2)
+    h = len(x) // 2
+    return _add(_pairwise(x[:h]), _pairwise(x[h:]))
+
+
+def _sequential(x):
+    acc = np.float32(0)
+    for v in x:
+        acc = _fma(v, acc)
+    return acc
+
+
+def _lane_order(p):
+    s = np.float32(0)
+    for v in p:
+        s = _add(s, v)
+    return s
+
+
+def test_sumsq_tree_golden_row():
+    """The page's tree (lane l owns 8-element chunks l, l+32, ...; fused
+    multiply-add in element order; butterfly 16...1) on the hand-worked row
+    gives 2^24 + 8; every other plausible order gives 2^24 + 4 or 2^24 + 12,
+    so the oracle fails this test under any of them."""
+    x, _, rec = sumsq_golden()
+    want = np.float32(int(rec["sumsq"]))
+    assert float(oracle.sumsq_tree(x)) == float(want)
+    rule = _butterfly(_lanes(x, 8, lambda c: c % 32))
+    assert rule == want  # the golden's own derivation
+    others = {
+        "sequential": _sequential(x),
+        "pairwise": _pairwise(list(x)),
+        "contiguous chunks per lane": _butterfly(_lanes(x, 8, lambda c: c // 2)),
+        "1-element chunks": _butterfly(_lanes(x, 1, lambda c: c % 32)),
+        "4-element chunks": _butterfly(_lanes(x, 4, lambda c: c % 32)),
+        "16-element chunks": _butterfly(_lanes(x, 16, lambda c: c % 32)),
+        "butterfly 1..16": _butterfly(_lanes(x, 8, lambda c: c % 32), (1, 2, 4, 8, 16)),
+        "lane sums in lane order": _lane_order(_lanes(x, 8, lambda c: c % 32)),
+        "exact, rounded once": np.float32(math.fsum(float(v) ** 2 for v in x)),
+    }
+    same = [k for k, v in others.items() if v == want]
+    assert not same, f"the golden row does not separate the tree from {same}"
+
+
+def test_sumsq_tree_golden_fused_multiply_add():
+    """Inside a lane the squares accumulate with a fused multiply-add: the
+    hand-worked pair gives 0x1.01f1d2p+1, a multiply then an add gives
+    0x1.01f1d0p+1."""
+    _, xf, rec = sumsq_golden()
+    assert float(oracle.sumsq_tree(xf)) == float.fromhex(rec["fma_sum"])
+    sq = np.float32(np.float64(xf[1]) ** 2)
+    unfused = _add(np.float32(np.float64(xf[0]) ** 2), sq)
+    assert float(unfused) != float.fromhex(rec["fma_sum"])
+
+
+def test_rmsnorm_global_scale_golden_row():
+    """RMSNorm (gain 1 except gain[0]) then the NVFP4 global scale of the
+    golden row: the fp32 bits worked by hand in the golden file."""
+    x, _, rec = sumsq_golden()
+    xb = _bits_bf16(x)
+    gam = np.full(512, 0x3F80, np.uint16)
+    gam[0] = int(rec["gain0"], 16)
+    _, _, g = oracle.quantize_nvfp4(xb[None, :], gam, 1e-6, oracle.F_RMSNORM)
+    assert int(g.view(np.uint32)[0]) == int(rec["g_bits"], 16)
+
+
 # ------------------------------------------------------------- FP8
 def test_fp8_row_scale_and_bounds():
     rng = np.random.default_rng(12)
