@@ -62,10 +62,6 @@ def to_bits(t: torch.Tensor) -> np.ndarray:
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def from_bits(a: np.ndarray) -> torch.Tensor:
-    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint16).view(np.int16)).view(torch.bfloat16)
-
-
 def tiny_inputs(seed: int = 0):
     """X [16, 256] with two x20 outlier channels, W [128, 256] ~ N(0, 0.02^2)."""
     gx = _gen(seed, _S_X)
@@ -123,10 +119,3 @@ FUSED_CASES = [
 
 def stack_seed(layer: int, proj: int) -> int:
     return 1000 + 7 * layer + proj
-
-
-def random_small(M: int, N: int, K: int, seed: int, outliers: bool = True):
-    """Small seeded case for parity tests: X with lognormal channel scales."""
-    X = projection_activations(K, M, seed)
-    W = projection_weight(K, N, seed)
-    return X, W

@@ -78,6 +78,63 @@ def gemm_error(Y_gpu, Y64):
     return rel, float(np.abs(d).max())
 
 
+U32 = 2.0 ** -24  # fp32 unit roundoff
+
+
+def half_ulp_bf16(v):
+    """Half the bf16 spacing at |v| (8 significant bits; subnormal floor)."""
+    a = np.maximum(np.abs(v), 2.0 ** -126)
+    return np.ldexp(1.0, np.floor(np.log2(a)).astype(np.int64) - 8)
+
+
+def elementwise_bound(Y64, Y_gpu, absdot, K, residual=None):
+    """Per-element bound on |Y - Y64| for a GEMM that accumulates in fp32
+    and rounds its output to bf16 once:
+      1/2 ulp_bf16 of the larger of |Y|, |Y64|        (output rounding)
+      + K u sum_k |x_k w_k|                           (at most K fp32 additions
+                                                       in the accumulation
+                                                       chain, split-K partials
+                                                       included: gamma_K <= K u
+                                                       to first order)
+      + 4 u (sum_k |x_k w_k| + |residual|)            (global-scale product,
+                                                       scaling, residual add)
+    with u = 2^-24 and x, w the decoded operands (absdot = |X| |W|^T)."""
+    bound = half_ulp_bf16(np.maximum(np.abs(Y64), np.abs(Y_gpu.astype(np.float64))))
+    bound = bound + (K + 4) * U32 * absdot
+    if residual is not None:
+        bound = bound + 4 * U32 * np.abs(residual)
+    return bound
+
+
+def check_gemm(Y_gpu, Y64, dx, dw, K, residual=None, what=""):
+    """Relative Frobenius gate (< REL_FRO_TOL) and the element-wise bound on
+    every compared element.  dx [rows, K], dw [N, K] are the decoded
+    operands of exactly the compared rows; residual (fp64 [rows, N]) or
+    None.  Returns (rel_fro, max_abs, worst error / bound)."""
+    Yg = Y_gpu.astype(np.float64)
+    rel, mx = gemm_error(Yg, Y64)
+    absdot = np.abs(np.asarray(dx, np.float64)) @ np.abs(np.asarray(dw, np.float64)).T
+    bound = elementwise_bound(Y64, Yg, absdot, K, residual)
+    ratio = np.abs(Yg - Y64) / bound
+    worst = float(ratio.max()) if ratio.size else 0.0
+    print(f"{what}: rel_fro={rel:.3e} max_abs={mx:.3e} worst err/bound={worst:.3f}")
+    assert np.isfinite(Yg).all(), f"{what}: non-finite output"
+    assert rel < REL_FRO_TOL, (what, rel, mx)
+    if worst > 1.0:
+        i = np.unravel_index(int(ratio.argmax()), ratio.shape)
+        raise AssertionError(f"{what}: element {tuple(int(t) for t in i)} off by {abs(Yg[i] - Y64[i]):.4e} "
+                             f"> bound {bound[i]:.4e} (Y={Yg[i]:.6e}, Y64={Y64[i]:.6e})")
+    return rel, mx, worst
+
+
+def residual_f64(R_bf16, rows=None):
+    """bf16 residual tensor -> fp64 numpy (optionally a row subset)."""
+    if R_bf16 is None:
+        return None
+    r = R_bf16.float().cpu().numpy().astype(np.float64)
+    return r if rows is None else r[rows]
+
+
 def gpu_linear_nvfp4(xq, xs, gx, wq, ws, gw, M, N, K, residual=None):
     """Device tensors in the library layouts -> Y (bf16, host numpy fp32)."""
     m = vq()

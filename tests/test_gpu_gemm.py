@@ -3,8 +3,11 @@
 The GEMM is fed the oracle's own codes and scales (re-laid out into the
 library's padded / tiled buffers), so the comparison isolates the GEMM; the
 end-to-end cases run the GPU quantizers too (their bytes are bit-exact, see
-test_gpu_quant.py).  Gate: relative Frobenius error < 2e-3 against the fp64
-result on the same decoded operands; max-abs is reported."""
+test_gpu_quant.py).  Gates, on every output element: relative Frobenius
+error < 2e-3 against the fp64 result on the same decoded operands, and the
+element-wise bound of an fp32-accumulated GEMM with one bf16 output rounding
+(gpu_helpers.elementwise_bound); max-abs and the worst error / bound ratio
+are printed."""
 import numpy as np
 import pytest
 import torch
@@ -12,8 +15,8 @@ import torch
 import layouts
 import oracle
 import synthetic_inputs as si
-from gpu_helpers import (REL_FRO_TOL, bits, gemm_error, gpu_linear_fp8, gpu_linear_nvfp4,
-                         gpu_quant_act_nvfp4, gpu_quant_weight_nvfp4, to_dev, vq)
+from gpu_helpers import (REL_FRO_TOL, bits, check_gemm, gemm_error, gpu_linear_fp8, gpu_linear_nvfp4,
+                         gpu_quant_act_nvfp4, gpu_quant_weight_nvfp4, residual_f64, to_dev, vq)
 
 pytestmark = pytest.mark.gpu
 
@@ -27,11 +30,16 @@ def _oracle_case(M, N, K, seed, residual=False, flags=0):
     dx = oracle.decode_nvfp4(cx, sx, gx, K)
     dw = oracle.decode_nvfp4(cw, sw, gw, K, per_tensor=True)
     Y64 = oracle.linear_f64(dx, dw, None if R is None else bits(R))
-    return (cx, sx, gx, cw, sw, gw, R, Y64)
+    return (cx, sx, gx, cw, sw, gw, R, Y64, dx, dw)
+
+
+def _check(Y, case, K, what):
+    """Frobenius gate and the element-wise bound against the oracle case."""
+    return check_gemm(Y, case[7], case[8], case[9], K, residual_f64(case[6]), what)
 
 
 def _run_nvfp4_from_oracle(M, N, K, case):
-    cx, sx, gx, cw, sw, gw, R, _ = case
+    cx, sx, gx, cw, sw, gw, R = case[:7]
     return gpu_linear_nvfp4(to_dev(layouts.pad_codes(cx, K)), to_dev(layouts.tile_scales(sx, M, K)), to_dev(gx),
                             to_dev(layouts.pad_codes(cw, K)), to_dev(layouts.tile_scales(sw, N, K)), to_dev(gw),
                             M, N, K, None if R is None else R.cuda())
@@ -60,9 +68,7 @@ NVFP4_CASES = [
 def test_linear_nvfp4_vs_oracle(M, N, K, res):
     case = _oracle_case(M, N, K, 21, residual=res)
     Y = _run_nvfp4_from_oracle(M, N, K, case)
-    rel, mx = gemm_error(Y, case[-1])
-    print(f"nvfp4 M={M} N={N} K={K} res={res}: rel_fro={rel:.3e} max_abs={mx:.3e}")
-    assert rel < REL_FRO_TOL, (rel, mx)
+    _check(Y, case, K, f"nvfp4 M={M} N={N} K={K} res={res}")
 
 
 def test_linear_nvfp4_single_element_parity_positions():
@@ -78,11 +84,11 @@ def test_linear_nvfp4_single_element_parity_positions():
         Wb = torch.from_numpy(w).to(torch.bfloat16)
         cx, sx, gx = oracle.quantize_nvfp4(bits(Xb))
         cw, sw, gw = oracle.quantize_nvfp4(bits(Wb), per_tensor=True)
-        Y64 = oracle.linear_f64(oracle.decode_nvfp4(cx, sx, gx, K),
-                                oracle.decode_nvfp4(cw, sw, gw, K, per_tensor=True))
-        Y = _run_nvfp4_from_oracle(M, N, K, (cx, sx, gx, cw, sw, gw, None, Y64))
-        rel, _ = gemm_error(Y, Y64)
-        assert rel < REL_FRO_TOL, (pos, rel)
+        dx = oracle.decode_nvfp4(cx, sx, gx, K)
+        dw = oracle.decode_nvfp4(cw, sw, gw, K, per_tensor=True)
+        case = (cx, sx, gx, cw, sw, gw, None, oracle.linear_f64(dx, dw), dx, dw)
+        Y = _run_nvfp4_from_oracle(M, N, K, case)
+        _check(Y, case, K, f"single element at {pos}")
 
 
 @pytest.mark.parametrize("M,N,K,res", [(16, 128, 256, False), (300, 392, 1024, True), (129, 136, 208, False),
@@ -93,11 +99,10 @@ def test_linear_fp8_vs_oracle(M, N, K, res):
     cx, sx = oracle.quantize_fp8(bits(X))
     cw, sw = oracle.quantize_fp8(bits(W))
     R = si.residual(M, N, 31) if res else None
-    Y64 = oracle.linear_f64(oracle.decode_fp8(cx, sx), oracle.decode_fp8(cw, sw), None if R is None else bits(R))
+    dx, dw = oracle.decode_fp8(cx, sx), oracle.decode_fp8(cw, sw)
+    Y64 = oracle.linear_f64(dx, dw, None if R is None else bits(R))
     Y = gpu_linear_fp8(to_dev(cx), to_dev(sx), to_dev(cw), to_dev(sw), M, N, K, None if R is None else R.cuda())
-    rel, mx = gemm_error(Y, Y64)
-    print(f"fp8 M={M} N={N} K={K}: rel_fro={rel:.3e} max_abs={mx:.3e}")
-    assert rel < REL_FRO_TOL, (rel, mx)
+    check_gemm(Y, Y64, dx, dw, K, residual_f64(R), f"fp8 M={M} N={N} K={K} res={res}")
 
 
 @pytest.mark.parametrize("M,N,K,flags,res", [(200, 256, 1024, 0, False), (70, 384, 512, 3, True),
@@ -111,15 +116,15 @@ def test_end_to_end_nvfp4(M, N, K, flags, res):
     R = si.residual(M, N, 41) if res else None
     cx, sx, gx = oracle.quantize_nvfp4(bits(X), bits(gam), 1e-6, flags)
     cw, sw, gw = oracle.quantize_nvfp4(bits(W), flags=flags & 2, per_tensor=True)
-    Y64 = oracle.linear_f64(oracle.decode_nvfp4(cx, sx, gx, K), oracle.decode_nvfp4(cw, sw, gw, K, per_tensor=True),
-                            None if R is None else bits(R))
+    dx = oracle.decode_nvfp4(cx, sx, gx, K)
+    dw = oracle.decode_nvfp4(cw, sw, gw, K, per_tensor=True)
+    Y64 = oracle.linear_f64(dx, dw, None if R is None else bits(R))
     xq, xs, xg = m.alloc_nvfp4(M, K)
     wq, ws, wg = m.alloc_nvfp4(N, K, per_tensor=True)
     m.vlaq_quantize_weight_nvfp4(W.cuda(), N, K, flags & 2, wq, ws, wg)
     m.vlaq_quantize_act_nvfp4(X.cuda(), M, K, gam.cuda(), 1e-6, flags, xq, xs, xg)
     Y = gpu_linear_nvfp4(xq, xs, xg, wq, ws, wg, M, N, K, None if R is None else R.cuda())
-    rel, mx = gemm_error(Y, Y64)
-    assert rel < REL_FRO_TOL, (rel, mx)
+    check_gemm(Y, Y64, dx, dw, K, residual_f64(R), f"end to end M={M} N={N} K={K} flags={flags}")
 
 
 def test_workspace_is_checked():
@@ -150,9 +155,7 @@ def test_linear_nvfp4_wide_tiles_vs_oracle(M, N, K, res):
     assert m.vlaq_linear_workspace_bytes(M, N, K) == 0
     case = _oracle_case(M, N, K, 23, residual=res)
     Y = _run_nvfp4_from_oracle(M, N, K, case)
-    rel, mx = gemm_error(Y, case[-1])
-    print(f"nvfp4 wide M={M} N={N} K={K} res={res}: rel_fro={rel:.3e} max_abs={mx:.3e}")
-    assert rel < REL_FRO_TOL, (rel, mx)
+    _check(Y, case, K, f"nvfp4 wide M={M} N={N} K={K} res={res}")
 
 
 @pytest.mark.parametrize("M,N,K,res", WIDE_CASES[:2])
@@ -162,10 +165,10 @@ def test_linear_fp8_wide_tiles_vs_oracle(M, N, K, res):
     cx, sx = oracle.quantize_fp8(bits(X))
     cw, sw = oracle.quantize_fp8(bits(W))
     R = si.residual(M, N, 33) if res else None
-    Y64 = oracle.linear_f64(oracle.decode_fp8(cx, sx), oracle.decode_fp8(cw, sw), None if R is None else bits(R))
+    dx, dw = oracle.decode_fp8(cx, sx), oracle.decode_fp8(cw, sw)
+    Y64 = oracle.linear_f64(dx, dw, None if R is None else bits(R))
     Y = gpu_linear_fp8(to_dev(cx), to_dev(sx), to_dev(cw), to_dev(sw), M, N, K, None if R is None else R.cuda())
-    rel, mx = gemm_error(Y, Y64)
-    assert rel < REL_FRO_TOL, (rel, mx)
+    check_gemm(Y, Y64, dx, dw, K, residual_f64(R), f"fp8 wide M={M} N={N} K={K} res={res}")
 
 
 def test_split_workspace_reused_across_calls_and_shapes():
@@ -180,7 +183,7 @@ def test_split_workspace_reused_across_calls_and_shapes():
     wsp = torch.zeros(need, dtype=torch.uint8, device="cuda")
     cases = {s: _oracle_case(*s, 51) for s in shapes}
     dev = {}
-    for (M, N, K), (cx, sx, gx, cw, sw, gw, _, _) in cases.items():
+    for (M, N, K), (cx, sx, gx, cw, sw, gw, *_) in cases.items():
         dev[(M, N, K)] = (to_dev(layouts.pad_codes(cx, K)), to_dev(layouts.tile_scales(sx, M, K)), to_dev(gx),
                           to_dev(layouts.pad_codes(cw, K)), to_dev(layouts.tile_scales(sw, N, K)), to_dev(gw))
     first = {}
@@ -191,8 +194,7 @@ def test_split_workspace_reused_across_calls_and_shapes():
             torch.cuda.synchronize()
             m.vlaq_check()
             y = Y.float().cpu().numpy()
-            rel, mx = gemm_error(y, cases[(M, N, K)][-1])
-            assert rel < REL_FRO_TOL, (rep, M, N, K, rel, mx)
+            _check(y, cases[(M, N, K)], K, f"rep {rep} {M}x{N}x{K}")
             if rep == 0:
                 first[(M, N, K)] = y
             else:
@@ -217,14 +219,13 @@ def test_linear_nvfp4_few_rows(M, N, K, res):
     cx, sx, gx = oracle.quantize_nvfp4(bits(X))
     cw, sw, gw = oracle.quantize_nvfp4(bits(W), per_tensor=True)
     R = si.residual(M, N, 61) if res else None
-    Y64 = oracle.linear_f64(oracle.decode_nvfp4(cx, sx, gx, K), oracle.decode_nvfp4(cw, sw, gw, K, per_tensor=True),
-                            None if R is None else bits(R))
+    dx = oracle.decode_nvfp4(cx, sx, gx, K)
+    dw = oracle.decode_nvfp4(cw, sw, gw, K, per_tensor=True)
+    Y64 = oracle.linear_f64(dx, dw, None if R is None else bits(R))
     dev = (to_dev(layouts.pad_codes(cx, K)), to_dev(layouts.tile_scales(sx, M, K)), to_dev(gx),
            to_dev(layouts.pad_codes(cw, K)), to_dev(layouts.tile_scales(sw, N, K)), to_dev(gw))
     Y = gpu_linear_nvfp4(*dev, M, N, K, None if R is None else R.cuda())
-    rel, mx = gemm_error(Y, Y64)
-    print(f"few rows M={M} N={N} K={K}: rel_fro={rel:.3e} max_abs={mx:.3e}")
-    assert rel < REL_FRO_TOL, (rel, mx)
+    check_gemm(Y, Y64, dx, dw, K, residual_f64(R), f"few rows M={M} N={N} K={K} res={res}")
     # the CUDA-core kernel needs no workspace; a second call gives the same bits
     few = M <= 2 and N * K <= 1 << 25
     Y2 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
