@@ -234,6 +234,17 @@ VLAQ_API size_t vlaq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *   Y            out, bf16 [M, N]
  *   workspace    device buffer of ws_bytes >= vlaq_linear_workspace_bytes
  * M == 0 is a no-op.  Limits: 1 <= N, 16 <= K, K % 16 == 0, N % 8 == 0.
+ * Stream order: the kernel is launched with programmatic dependent launch
+ * and starts streaming the weight operand (wq, ws) before it waits for the
+ * kernel launched just before it on the same stream; everything else
+ * (activations, globals, residual, workspace, Y) is touched only after that
+ * wait.  So wq and ws must not be written by the kernel launched
+ * immediately before this call on the stream.  Every kernel two or more
+ * launches back has completed by then (each library kernel lets its
+ * successor start only after its own wait), so weights produced by
+ * vlaq_quantize_weight_nvfp4 right before this call are safe: its codes and
+ * scales come from its second-to-last kernel, its last kernel writes g_w
+ * only, and g_w is read after the wait.
  * (Residual add in the o / down epilogues: "FoldQuant W8A8/W4A4 inference",
  * merge commit.) */
 VLAQ_API vlaq_status vlaq_linear_nvfp4(const uint8_t* xq, const uint8_t* xs,
@@ -250,9 +261,11 @@ VLAQ_API vlaq_status vlaq_linear_nvfp4(const uint8_t* xq, const uint8_t* xs,
  * The split-K partial sums of small-M shapes go to a 4 MiB array compiled
  * into the library, which every GPU that loads the library holds until the
  * process exits.  A shape whose split-K plan needs more than 4 MiB is refused
- * with VLAQ_ERR_WORKSPACE (use vlaq_linear_nvfp4 then).  The first call on
- * each device looks the array's address up (cudaGetSymbolAddress) and caches
- * it; make that first call before any stream capture.  All calls on a
+ * with VLAQ_ERR_WORKSPACE (use vlaq_linear_nvfp4 then).  The first call
+ * that needs the array in a CUDA context (one per device; a new one after
+ * cudaDeviceReset) looks its address up (cudaGetSymbolAddress) with that
+ * device current and caches it beside the context's ID; make that first
+ * call before any stream capture.  All calls on a
  * device share the array (zero when the library loads; each call leaves its
  * tile counters zero again, and vlaq_check clears the array when it
  * reports VLAQ_ERR_TIMEOUT); calls that overlap on the GPU, e.g. on two

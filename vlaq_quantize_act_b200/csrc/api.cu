@@ -327,9 +327,12 @@ size_t vlaq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
 
 enum LinearKind { kLinearNvfp4, kLinearFp8, kLinearInt8 };
 
+// static_scratch: the split-K scratch is the library's static array
+// (vlaq_linear_nvfp4_noalloc) instead of the caller's workspace.
 static vlaq_status linear_common(const char* fn, LinearKind kind, const uint8_t* xq, const uint8_t* xs, const float* xg,
                                  const uint8_t* wq, const uint8_t* ws, const float* wg, const void* residual, void* Y,
-                                 int64_t M, int64_t N, int64_t K, void* workspace, size_t ws_bytes, void* stream) {
+                                 int64_t M, int64_t N, int64_t K, void* workspace, size_t ws_bytes, void* stream,
+                                 bool static_scratch = false) {
   vlaq_status st;
   const bool fp4 = kind == kLinearNvfp4;
   if ((st = check_k(fn, K, 0, fp4, 0))) return st;
@@ -352,6 +355,16 @@ static vlaq_status linear_common(const char* fn, LinearKind kind, const uint8_t*
   if (residual && !aligned16(residual)) return fail(VLAQ_ERR_ALIGN, "%s: residual is not 16-byte aligned", fn);
   if ((st = check_device(fn))) return st;
   const vlaq::GemmPlan plan = vlaq::plan_gemm(fp4, M, N, K, vlaq::device_sm_count());
+  if (static_scratch && plan.ws_bytes > 0) {
+    if (plan.ws_bytes > vlaq::kNoallocScratchBytes)
+      return fail(VLAQ_ERR_WORKSPACE,
+                  "%s: shape %lld x %lld x %lld needs %zu bytes of split-K scratch, more than the %zu-byte static "
+                  "scratch array; use vlaq_linear_nvfp4 with a caller-allocated workspace",
+                  fn, (long long)M, (long long)N, (long long)K, plan.ws_bytes, vlaq::kNoallocScratchBytes);
+    cudaError_t e = vlaq::noalloc_scratch(&workspace);
+    if (e != cudaSuccess) return cuda_fail(fn, e);
+    ws_bytes = vlaq::kNoallocScratchBytes;
+  }
   if (plan.ws_bytes > 0) {
     if (!workspace || ws_bytes < plan.ws_bytes)
       return fail(VLAQ_ERR_WORKSPACE, "%s: this shape needs %zu bytes of workspace (got %zu%s)", fn, plan.ws_bytes,
@@ -394,26 +407,10 @@ vlaq_status vlaq_linear_int8(const int8_t* xq, const float* s_x, const int8_t* w
 vlaq_status vlaq_linear_nvfp4_noalloc(const uint8_t* xq, const uint8_t* xs, const float* g_x, const uint8_t* wq,
                                       const uint8_t* ws, const float* g_w, const void* residual, void* Y, int64_t M,
                                       int64_t N, int64_t K, void* stream) {
-  const char* fn = "vlaq_linear_nvfp4_noalloc";
-  // Shapes the regular validation accepts get their scratch need checked
-  // against the fixed array; everything else is refused by linear_common
-  // with the usual messages.
-  if (M > 0 && N > 0 && N % 8 == 0 && K > 0 && K % 16 == 0 && M <= 0x7FFFFFFF && N <= 0x7FFFFFFF &&
-      K <= 0x7FFFFFFF) {
-    const size_t need = vlaq::plan_gemm(true, M, N, K, vlaq::device_sm_count()).ws_bytes;
-    if (need > vlaq::kNoallocScratchBytes)
-      return fail(VLAQ_ERR_WORKSPACE,
-                  "%s: shape %lld x %lld x %lld needs %zu bytes of split-K scratch, more than the %zu-byte static "
-                  "scratch array; use vlaq_linear_nvfp4 with a caller-allocated workspace",
-                  fn, (long long)M, (long long)N, (long long)K, need, vlaq::kNoallocScratchBytes);
-  }
-  void* scratch = nullptr;
-  if (M > 0) {
-    cudaError_t e = vlaq::noalloc_scratch(&scratch);
-    if (e != cudaSuccess) return cuda_fail(fn, e);
-  }
-  return linear_common(fn, kLinearNvfp4, xq, xs, g_x, wq, ws, g_w, residual, Y, M, N, K, scratch,
-                       vlaq::kNoallocScratchBytes, stream);
+  // same validation and order as vlaq_linear_nvfp4; a split-K plan takes the
+  // library's static scratch array (refused if it needs more)
+  return linear_common("vlaq_linear_nvfp4_noalloc", kLinearNvfp4, xq, xs, g_x, wq, ws, g_w, residual, Y, M, N, K,
+                       nullptr, 0, stream, true);
 }
 
 }  // extern "C"
