@@ -17,11 +17,22 @@ Reported (one JSON line on rank 0):
              its stream: algorithmic FLOPs / launch duration vs the measured
              dense FP4 peak (bf16 burst peak x 4, the nominal FP4:BF16 ratio)
   prologue   the activation prologue: algorithmic bytes / duration vs HBM
-  decode     M = 1 (weight-bandwidth-bound): GB/s of algorithmic bytes,
-             weights rotated over two copies so the working set exceeds L2
-  fp8, int8  the FP8 and INT8 W8A8 variants of the same step (TFLOP/s; INT8
-             multiply-accumulates counted as FLOPs)
-  cpu_baseline  the CPU oracle on a bounded sample of the same workload
+  decode     M = 1, 4, 8 (weight-bandwidth-bound): GB/s of algorithmic
+             bytes, weights rotated over copies so the working set exceeds L2
+  fused      the fused-prologue step (RMSNorm + block-64 rotation on the
+             qkv / gate_up inputs, rotation + residual add on o / down,
+             rotated weights), NVFP4 and FP8 W8A8
+  fp8, int8  the FP8 and INT8 W8A8 variants of the plain step (TFLOP/s;
+             INT8 multiply-accumulates counted as FLOPs)
+  stack      the 28-layer stack (196 projections, one graph), all NVFP4 and
+             mixed (o / down FP8), at M = 1024 and M = 1: us per token
+  cpu_baseline  the CPU oracle on a bounded sample of the same workload,
+             with one entry per workload above
+Kernel durations: CUDA events recorded as nodes inside the captured step
+("in_step": includes the node-to-node launch gap, which is a large share of
+a few-microsecond kernel), and for the prologue and the decode GEMMs also a
+graph of the same kernel launched back to back over buffers larger than L2
+("back_to_back": per-launch time in a stream of such launches).
 Inputs: seeded synthetic bf16 (synthetic_inputs.py); the per-step working set
 (X 61 MB + W 131 MB + Y 102 MB) exceeds the 126 MB L2.
 
@@ -163,32 +174,44 @@ def make_inputs(M, device, seed_offset=0):
     return data
 
 
-class Step:
-    """Device buffers and launch sequence of one hot-path step."""
+FUSED = {c.name: c for c in si.FUSED_CASES}
 
-    def __init__(self, vq, data, M, device, fmt="nvfp4", weight_copies=1):
+
+class Step:
+    """Device buffers and launch sequence of one hot-path step.  fused: the
+    fused-prologue workload (RMSNorm + block-64 rotation on the qkv /
+    gate_up inputs, rotation only plus a residual add on o / down, weights
+    rotated too)."""
+
+    def __init__(self, vq, data, M, device, fmt="nvfp4", weight_copies=1, fused=False):
         assert fmt in ("nvfp4", "fp8", "int8"), fmt
         self.vq = vq
         self.M = M
         self.fmt = fmt
         self.fp8 = fmt != "nvfp4"  # an 8-bit W8A8 format (FP8 or INT8)
+        self.fused = fused
         self.layers = []
         for name in PROJ:
             K, N, X, W = data[name]
+            case = FUSED[name]
+            flags = (3 if case.rmsnorm else 2) if fused else 0
+            wflags = flags & 2
             Wd = W.to(device)
             copies = []
-            for _ in range(weight_copies):
-                if fmt == "fp8":
+            for c in range(weight_copies):
+                if c > 0:  # further copies: the same bytes in other buffers
+                    copies.append(tuple(None if t is None else t.clone() for t in copies[0]))
+                elif fmt == "fp8":
                     wq, sw = vq.alloc_fp8(N, K, device)
-                    vq.vlaq_quantize_weight_fp8(Wd, N, K, 0, wq, sw)
+                    vq.vlaq_quantize_weight_fp8(Wd, N, K, wflags, wq, sw)
                     copies.append((wq, None, sw))
                 elif fmt == "int8":
                     wq, sw = vq.alloc_int8(N, K, device)
-                    vq.vlaq_quantize_weight_int8(Wd, N, K, 0, wq, sw)
+                    vq.vlaq_quantize_weight_int8(Wd, N, K, wflags, wq, sw)
                     copies.append((wq, None, sw))
                 else:
                     wq, ws, wg = vq.alloc_nvfp4(N, K, device, per_tensor=True)
-                    vq.vlaq_quantize_weight_nvfp4(Wd, N, K, 0, wq, ws, wg)
+                    vq.vlaq_quantize_weight_nvfp4(Wd, N, K, wflags, wq, ws, wg)
                     copies.append((wq, ws, wg))
             del Wd
             Xd = X.to(device)
@@ -199,42 +222,53 @@ class Step:
                 act = vq.alloc_nvfp4(M, K, device)
             Y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
             wsp, nb = vq.alloc_workspace(M, N, K, device)
-            self.layers.append(dict(name=name, K=K, N=N, X=Xd, act=act, W=copies, Y=Y, ws=wsp, nb=nb))
+            gam = si.norm_gain(K, FUSED[name].seed).to(device) if flags & 1 else None
+            R = si.residual(M, N, FUSED[name].seed).to(device) if fused and case.residual else None
+            self.layers.append(dict(name=name, K=K, N=N, X=Xd, act=act, W=copies, Y=Y, ws=wsp, nb=nb,
+                                    flags=flags, gamma=gam, R=R))
         torch.cuda.synchronize()
         self.flops = sum(2.0 * M * L["N"] * L["K"] for L in self.layers)
 
     def run(self, copy=0, events=None):
-        vq = self.vq
-        M = self.M
         for i, L in enumerate(self.layers):
-            K, N = L["K"], L["N"]
-            xq, xs, xg = L["act"]
-            wq, ws, wg = L["W"][copy % len(L["W"])]
             if events is not None:
                 events[i][0].record()
-            if self.fmt == "fp8":
-                vq.vlaq_quantize_act_fp8(L["X"], M, K, None, 1e-6, 0, xq, xg)
-            elif self.fmt == "int8":
-                vq.vlaq_quantize_act_int8(L["X"], M, K, None, 1e-6, 0, xq, xg)
-            else:
-                vq.vlaq_quantize_act_nvfp4(L["X"], M, K, None, 1e-6, 0, xq, xs, xg)
+            self.prologue(L)
             if events is not None:
                 events[i][1].record()
-            if self.fmt == "fp8":
-                vq.vlaq_linear_fp8(xq, xg, wq, wg, None, L["Y"], M, N, K, L["ws"], L["nb"])
-            elif self.fmt == "int8":
-                vq.vlaq_linear_int8(xq, xg, wq, wg, None, L["Y"], M, N, K, L["ws"], L["nb"])
-            else:
-                vq.vlaq_linear_nvfp4(xq, xs, xg, wq, ws, wg, None, L["Y"], M, N, K, L["ws"], L["nb"])
+            self.gemm(L, copy)
             if events is not None:
                 events[i][2].record()
 
+    def prologue(self, L, X=None):
+        vq, M, K = self.vq, self.M, L["K"]
+        X = L["X"] if X is None else X
+        xq, xs, xg = L["act"]
+        if self.fmt == "fp8":
+            vq.vlaq_quantize_act_fp8(X, M, K, L["gamma"], 1e-6, L["flags"], xq, xg)
+        elif self.fmt == "int8":
+            vq.vlaq_quantize_act_int8(X, M, K, L["gamma"], 1e-6, L["flags"], xq, xg)
+        else:
+            vq.vlaq_quantize_act_nvfp4(X, M, K, L["gamma"], 1e-6, L["flags"], xq, xs, xg)
+
+    def gemm(self, L, copy=0):
+        vq, M, K, N = self.vq, self.M, L["K"], L["N"]
+        xq, xs, xg = L["act"]
+        wq, ws, wg = L["W"][copy % len(L["W"])]
+        if self.fmt == "fp8":
+            vq.vlaq_linear_fp8(xq, xg, wq, wg, L["R"], L["Y"], M, N, K, L["ws"], L["nb"])
+        elif self.fmt == "int8":
+            vq.vlaq_linear_int8(xq, xg, wq, wg, L["R"], L["Y"], M, N, K, L["ws"], L["nb"])
+        else:
+            vq.vlaq_linear_nvfp4(xq, xs, xg, wq, ws, wg, L["R"], L["Y"], M, N, K, L["ws"], L["nb"])
+
     def gemm_bytes(self, L):
-        """Algorithmic HBM bytes of one GEMM launch."""
+        """Algorithmic HBM bytes of one GEMM launch (residual read included)."""
         M, N, K = self.M, L["N"], L["K"]
+        res = 2 * M * N if L["R"] is not None else 0
         if self.fp8:
-            return N * K + 4 * N + M * K + 4 * M + 2 * M * N
-        return N * K // 2 + N * K // 16 + 4 + M * K // 2 + M * K // 16 + 4 * M + 2 * M * N
+            return N * K + 4 * N + M * K + 4 * M + 2 * M * N + res
+        return N * K // 2 + N * K // 16 + 4 + M * K // 2 + M * K // 16 + 4 * M + 2 * M * N + res
 
     def prologue_bytes(self, L):
         M, K = self.M, L["K"]
@@ -247,14 +281,19 @@ class Step:
 MIXED_FP8 = ("o", "down")
 
 
-def stack_weights(vq, device, layers=si.STACK_LAYERS, fp8=()):
+def stack_weights(vq, device, layers=si.STACK_LAYERS, fp8=(), reuse=None):
     """Weights of the 28-layer stack in (layer, projection) order, each
     quantized on the device right after it is generated (only the quantized
     copy stays: about 3.7 GB all NVFP4).  Projections named in fp8 get FP8
-    codes and per-row scales (2-tuples), the others NVFP4 (3-tuples)."""
+    codes and per-row scales (2-tuples), the others NVFP4 (3-tuples).
+    reuse: an all-NVFP4 list from an earlier call whose NVFP4 entries are
+    shared instead of regenerated."""
     out = []
     for l in range(layers):
         for p, (name, K, N) in enumerate(si.STACK_PROJECTIONS):
+            if reuse is not None and name not in fp8:
+                out.append(reuse[7 * l + p])
+                continue
             W = si.projection_weight(K, N, si.stack_seed(l, p)).to(device)
             if name in fp8:
                 wq, sw = vq.alloc_fp8(N, K, device)
@@ -512,6 +551,370 @@ def run_reference(args, rank):
     print(json.dumps(out), flush=True)
 
 
+class Launches:
+    """run() issues the given launches in order (a graph of them is timed
+    back to back)."""
+
+    def __init__(self, fns):
+        self.fns = fns
+
+    def run(self, c=0):
+        for f in self.fns:
+            f()
+
+
+def back_to_back_ms(fns, reps, warmup, dist_on, device):
+    """Per-launch time of `fns` launched back to back in one graph."""
+    g = capture(Launches(fns))
+    for _ in range(warmup):
+        g.replay()
+    ms = time_graph(g, reps, dist_on, device) / len(fns)
+    del g
+    return ms
+
+
+L2_BYTES = 126 * 2 ** 20
+
+
+def copies_beyond_l2(nbytes, least=2):
+    """Buffer copies whose total exceeds L2 (so every launch reads HBM)."""
+    return max(least, -(-int(1.25 * L2_BYTES) // max(int(nbytes), 1)))
+
+
+def prologue_back_to_back(step, args, dist_on, device):
+    """Per-projection prologue launch time, back to back over input copies
+    larger than L2 in total (ms)."""
+    out = {}
+    for L in step.layers:
+        xb = L["X"].numel() * L["X"].element_size()
+        Xs = [L["X"]] + [L["X"].clone() for _ in range(copies_beyond_l2(xb) - 1)]
+        fns = [(lambda X=X, L=L: step.prologue(L, X)) for X in Xs]
+        out[L["name"]] = back_to_back_ms(fns, args.steps, args.warmup, dist_on, device)
+        del Xs
+    return out
+
+
+def gemm_back_to_back(step, args, dist_on, device):
+    """Per-projection GEMM launch time, back to back over weight copies
+    larger than L2 in total (ms)."""
+    out = {}
+    for L in step.layers:
+        wb = sum(t.numel() * t.element_size() for t in L["W"][0] if t is not None)
+        need = copies_beyond_l2(wb)
+        extra = [tuple(None if t is None else t.clone() for t in L["W"][0]) for _ in range(need - len(L["W"]))]
+        W = L["W"] + extra
+        fns = []
+        for c in range(len(W)):
+            def f(c=c, L=L, W=W):
+                saved = L["W"]
+                L["W"] = W
+                step.gemm(L, c)
+                L["W"] = saved
+            fns.append(f)
+        out[L["name"]] = back_to_back_ms(fns, args.steps, args.warmup, dist_on, device)
+        del extra, W
+    return out
+
+
+def step_section(vq, step, args, dist_on, device, peaks, world, copies=1):
+    """Graph-timed step plus in-step kernel durations."""
+    graph = capture(step, copies)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    ms = time_graph(graph, args.steps, dist_on, device) / copies
+    del graph
+    pro, gem, tmode = kernel_durations(step, max(args.steps // 2, 3), copies=copies)
+    return ms, pro, gem, tmode
+
+
+def prefill_section(vq, data, args, dist_on, device, peaks, world):
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    step = Step(vq, data, M_PREFILL, device)
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    graph = capture(step)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    ms = time_graph(graph, args.steps, dist_on, device)
+    pro, gem, tmode = kernel_durations(step, max(args.steps // 2, 3))
+    clocks = sampler.stop()
+    del graph
+    value = world * step.flops / (ms / 1e3) / 1e12
+    # dominant kernel: the gate_up GEMM launch (about half of the step)
+    gi = PROJ.index("gate_up")
+    GL = step.layers[gi]
+    gu_ms = statistics.mean(gem[gi])
+    g_ach = 2.0 * M_PREFILL * GL["N"] * GL["K"] / (gu_ms / 1e3) / 1e12
+    gemm_all_ms = sum(statistics.mean(x) for x in gem)
+    gemm_all = step.flops / (gemm_all_ms / 1e3) / 1e12
+    pro_ms = sum(statistics.mean(x) for x in pro)
+    pro_bytes = sum(step.prologue_bytes(L) for L in step.layers)
+    b2b = prologue_back_to_back(step, args, dist_on, device)
+    b2b_ms = sum(b2b.values())
+    per_proj = {L["name"]: {"gemm_us": 1e3 * statistics.mean(gem[i]),
+                            "gemm_tflops": 2.0 * M_PREFILL * L["N"] * L["K"] / (statistics.mean(gem[i]) / 1e3) / 1e12,
+                            "prologue_us_in_step": 1e3 * statistics.mean(pro[i]),
+                            "prologue_us": 1e3 * b2b[L["name"]],
+                            "prologue_gbs": step.prologue_bytes(L) / (b2b[L["name"]] / 1e3) / 1e9}
+                for i, L in enumerate(step.layers)}
+    traffic = load_traffic("gemm_nvfp4_prefill")
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e2m1/e4m3 (fp32 accumulate, bf16 out)", "data": "synthetic",
+        "config": {"workload": "NVFP4 W4A4 prefill: act prologue + block-scaled FP4 GEMM for qkv 3584->4608, "
+                               "o 3584->3584, gate_up 3584->37888, down 18944->3584 (Qwen2.5-VL-7B shapes)",
+                   "global_batch": M_PREFILL * world, "seq_len": M_PREFILL, "parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2 (per-step working set ~294 MB)", "graph": True},
+        "roofline": {"bound": "tensor", "achieved": g_ach, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": g_ach / fp4_peak, "traffic": traffic,
+                     "kernel": "gemm_fp4_sfw_kernel gate_up 1024x37888x3584 (2MNK = 278.1 GFLOP per launch)",
+                     "all_gemms_tflops": gemm_all, "all_gemms_frac": gemm_all / fp4_peak,
+                     "timing": f"CUDA events in a {tmode} capture of the step",
+                     "peak_note": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 4 (nominal FP4:BF16)"},
+        "prologue": {"bound": "hbm", "achieved": pro_bytes / (b2b_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": pro_bytes / (b2b_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                     "achieved_in_step": pro_bytes / (pro_ms / 1e3) / 1e9,
+                     "frac_in_step": pro_bytes / (pro_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                     "kernel": "quant_rows_kernel (NVFP4 activation prologue), qkv / o / gate_up / down inputs",
+                     "timing": "achieved: back to back over input copies > L2 (per-launch time, CUDA events around "
+                               "the graph); in_step: event nodes around each launch inside the step"},
+        "per_projection": per_proj,
+        "clocks": clocks,
+    }
+    return step, out
+
+
+def decode_section(vq, data, args, dist_on, device, peaks, world):
+    """M = 1, 4, 8: the step over two weight copies, plus the GEMMs back to
+    back over weight copies larger than L2."""
+    res = {}
+    for M in (1, 4, 8):
+        ddata = {n: (K, N, X[:M].contiguous(), W) for n, (K, N, X, W) in data.items()}
+        dstep = Step(vq, ddata, M, device, weight_copies=2)
+        dms, dpro, dgem, _ = step_section(vq, dstep, args, dist_on, device, peaks, world, copies=2)
+        dbytes = sum(dstep.gemm_bytes(L) + dstep.prologue_bytes(L) for L in dstep.layers)
+        gem_bytes = {L["name"]: dstep.gemm_bytes(L) for L in dstep.layers}
+        b2b = gemm_back_to_back(dstep, args, dist_on, device)
+        tot_bytes = sum(gem_bytes.values())
+        b2b_ach = tot_bytes / (sum(b2b.values()) / 1e3) / 1e9
+        ins_ms = sum(sum(x) for x in dgem) / len(dgem[0])
+        res[str(M)] = {
+            "value": world * dbytes / (dms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": dms,
+            "bytes_per_step": dbytes, "M": M,
+            "gemm_roofline": {"bound": "hbm", "achieved": b2b_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                              "frac": b2b_ach / peaks["hbm_gbs"],
+                              "achieved_in_step": tot_bytes / (ins_ms / 1e3) / 1e9,
+                              "frac_in_step": tot_bytes / (ins_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                              "timing": "achieved: each GEMM back to back over weight copies > L2; in_step: "
+                                        "event nodes inside the step"},
+            "per_projection": {L["name"]: {"gemm_us": 1e3 * b2b[L["name"]],
+                                           "gemm_gbs": gem_bytes[L["name"]] / (b2b[L["name"]] / 1e3) / 1e9,
+                                           "gemm_us_in_step": 1e3 * statistics.mean(dgem[i]),
+                                           "prologue_us_in_step": 1e3 * statistics.mean(dpro[i])}
+                               for i, L in enumerate(dstep.layers)}}
+        del dstep
+        torch.cuda.empty_cache()
+    return res
+
+
+def w8a8_section(vq, data, args, dist_on, device, peaks, world, fmt, fused=False):
+    fstep = Step(vq, data, M_PREFILL, device, fmt=fmt, fused=fused)
+    fms, _, fgem, _ = step_section(vq, fstep, args, dist_on, device, peaks, world)
+    fgem_ms = sum(sum(x) for x in fgem) / len(fgem[0])
+    fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
+    out = {"value": world * fstep.flops / (fms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": fms,
+           "gemm_achieved": fstep.flops / (fgem_ms / 1e3) / 1e12, "peak": fp8_peak,
+           "frac": fstep.flops / (fgem_ms / 1e3) / 1e12 / fp8_peak}
+    del fstep
+    return out
+
+
+def fused_section(vq, data, args, dist_on, device, peaks, world):
+    """The fused-prologue step at M = 1024: NVFP4 and FP8 W8A8."""
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    step = Step(vq, data, M_PREFILL, device, fused=True)
+    ms, pro, gem, _ = step_section(vq, step, args, dist_on, device, peaks, world)
+    b2b = prologue_back_to_back(step, args, dist_on, device)
+    pro_bytes = sum(step.prologue_bytes(L) for L in step.layers)
+    gemm_ms = sum(statistics.mean(x) for x in gem)
+    out = {"nvfp4": {
+        "value": world * step.flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+        "gemm_tflops": step.flops / (gemm_ms / 1e3) / 1e12, "gemm_frac": step.flops / (gemm_ms / 1e3) / 1e12 / fp4_peak,
+        "prologue_gbs": pro_bytes / (sum(b2b.values()) / 1e3) / 1e9,
+        "prologue_frac": pro_bytes / (sum(b2b.values()) / 1e3) / 1e9 / peaks["hbm_gbs"],
+        "per_projection": {L["name"]: {"flags": L["flags"], "residual": L["R"] is not None,
+                                       "prologue_us": 1e3 * b2b[L["name"]],
+                                       "gemm_us_in_step": 1e3 * statistics.mean(gem[i])}
+                           for i, L in enumerate(step.layers)},
+        "workload": "RMSNorm (gain U(0.5,1.5), eps 1e-6) + block-64 WHT on qkv / gate_up inputs, WHT + residual "
+                    "add on o / down, WHT-rotated weights; M = 1024"}}
+    del step
+    out["fp8"] = w8a8_section(vq, data, args, dist_on, device, peaks, world, "fp8", fused=True)
+    return out
+
+
+def stack_section(vq, args, dist_on, device, world):
+    """28-layer stack, one graph of 196 prologue + GEMM pairs: all NVFP4,
+    then mixed (o / down FP8 W8A8, the rest NVFP4)."""
+    out = {}
+    sw = stack_weights(vq, device)
+    variants = (("", (), sw), ("mixed_", MIXED_FP8, None))
+    for prefix, fp8, w in variants:
+        if w is None:
+            w = stack_weights(vq, device, fp8=fp8, reuse=sw)
+        for sm in (M_PREFILL, 1):
+            st = Stack(vq, sm, device, weights=w, fp8=fp8)
+            sg = capture(st)
+            for _ in range(args.warmup):
+                sg.replay()
+            torch.cuda.synchronize()
+            sms = time_graph(sg, max(args.steps // 4, 3), dist_on, device)
+            key = prefix + ("prefill" if sm > 1 else "decode")
+            out[key] = {"M": sm, "ms": sms, "us_per_token": 1e3 * sms / sm,
+                        "tflops": world * st.flops / (sms / 1e3) / 1e12,
+                        "weight_gbs": world * st.weight_bytes / (sms / 1e3) / 1e9,
+                        "gemms": len(st.entries), "fp8_projections": list(fp8)}
+            del sg, st
+            torch.cuda.empty_cache()
+        del w
+    del sw
+    torch.cuda.empty_cache()
+    return out
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+class _OmpThreads:
+    """Sets the OpenMP thread count of this process (the oracle's GEMM is
+    parallel over output rows) for a single-core timing, then restores it."""
+
+    def __init__(self, n):
+        import ctypes
+        self.n = n
+        try:
+            self.lib = ctypes.CDLL("libgomp.so.1")
+        except OSError:
+            self.lib = None
+
+    def __enter__(self):
+        if self.lib:
+            self.prev = self.lib.omp_get_max_threads()
+            self.lib.omp_set_num_threads(self.n)
+        return self
+
+    def __exit__(self, *exc):
+        if self.lib:
+            self.lib.omp_set_num_threads(self.prev)
+
+
+def cpu_baselines(data, args):
+    """The CPU oracle, as it stands, on bounded samples of every workload."""
+    import oracle
+    cores = oracle.num_threads()
+    out = {"cores": cores, "cpu": cpu_model()}
+    # prefill: a token sample of each projection
+    t, fl, dec = cpu_oracle_sample(data, 1)
+    t, fl, _ = cpu_oracle_sample(data, args.cpu_rows, decoded_w=dec)
+    out["prefill"] = {"value": fl / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                      "sample": f"{args.cpu_rows} token rows of each projection: NVFP4 quantize + fp64 GEMM "
+                                f"({t:.1f} s)"}
+    # decode M = 1, 4, 8: every token, all four projections; GB/s of the
+    # same algorithmic bytes as the GPU line (the fp64 GEMM runs in parallel
+    # over output rows only, so M = 1 is one core)
+    dec_out = {}
+    for M in (1, 4, 8):
+        t0 = time.perf_counter()
+        nbytes = 0
+        for name in PROJ:
+            K, N, X, W = data[name]
+            cx, sx, gx = oracle.quantize_nvfp4(si.to_bits(X[:M]))
+            oracle.linear_f64(oracle.decode_nvfp4(cx, sx, gx, K), dec[name])
+            nbytes += N * K // 2 + N * K // 16 + M * K * 2 + 2 * M * N
+        tt = time.perf_counter() - t0
+        dec_out[str(M)] = {"value": nbytes / tt / 1e9, "unit": "GB/s", "s": tt,
+                           "cores": 1 if M == 1 else min(M, cores)}
+    out["decode"] = dec_out
+    # tiny workload (16 x 256 x 128), all cores and one core
+    X, W = si.tiny_inputs(0)
+    cw, sw, gw = oracle.quantize_nvfp4(si.to_bits(W), per_tensor=True)
+    dw = oracle.decode_nvfp4(cw, sw, gw, 256, per_tensor=True)
+
+    def tiny():
+        cx, sx, gx = oracle.quantize_nvfp4(si.to_bits(X))
+        oracle.linear_f64(oracle.decode_nvfp4(cx, sx, gx, 256), dw)
+
+    reps = 200
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        tiny()
+    ta = (time.perf_counter() - t0) / reps
+    with _OmpThreads(1):
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            tiny()
+        t1 = (time.perf_counter() - t0) / reps
+    out["tiny"] = {"unit": "GFLOP/s", "value": 2 * 16 * 128 * 256 / ta / 1e9, "single_core": 2 * 16 * 128 * 256 / t1 / 1e9,
+                   "us_per_call": 1e6 * ta, "us_per_call_single_core": 1e6 * t1}
+    # single-core decode M = 1 (as above, pinned to one thread)
+    with _OmpThreads(1):
+        t0 = time.perf_counter()
+        for name in PROJ:
+            K, N, X, W = data[name]
+            cx, sx, gx = oracle.quantize_nvfp4(si.to_bits(X[:1]))
+            oracle.linear_f64(oracle.decode_nvfp4(cx, sx, gx, K), dec[name])
+        out["decode"]["1"]["single_core_s"] = time.perf_counter() - t0
+    del dec
+    # fused workload: rotated weights, RMSNorm + rotation (qkv, gate_up) or
+    # rotation + residual (o, down) on a token sample
+    rows = max(args.cpu_rows // 16, 4)
+    t = fl = 0.0
+    for name in PROJ:
+        K, N, X, W = data[name]
+        case = FUSED[name]
+        flags = 3 if case.rmsnorm else 2
+        cw, sw, gw = oracle.quantize_nvfp4(si.to_bits(W), flags=2, per_tensor=True)
+        dw = oracle.decode_nvfp4(cw, sw, gw, K, per_tensor=True)
+        gam = si.to_bits(si.norm_gain(K, case.seed))
+        R = si.to_bits(si.residual(rows, N, case.seed)) if case.residual else None
+        t0 = time.perf_counter()
+        cx, sx, gx = oracle.quantize_nvfp4(si.to_bits(X[:rows]), gam, 1e-6, flags)
+        oracle.linear_f64(oracle.decode_nvfp4(cx, sx, gx, K), dw, R)
+        t += time.perf_counter() - t0
+        fl += 2.0 * rows * N * K
+        del dw
+    out["fused"] = {"value": fl / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                    "sample": f"{rows} token rows of each projection, fused prologue + fp64 GEMM ({t:.1f} s)"}
+    # 28-layer stack: layer 0 timed on a token sample, per token x 28 layers
+    rows = 4
+    t = 0.0
+    for p, (name, K, N) in enumerate(si.STACK_PROJECTIONS):
+        seed = si.stack_seed(0, p)
+        cw, sw, gw = oracle.quantize_nvfp4(si.to_bits(si.projection_weight(K, N, seed)), per_tensor=True)
+        dw = oracle.decode_nvfp4(cw, sw, gw, K, per_tensor=True)
+        X = si.projection_activations(K, rows, seed)
+        t0 = time.perf_counter()
+        cx, sx, gx = oracle.quantize_nvfp4(si.to_bits(X))
+        oracle.linear_f64(oracle.decode_nvfp4(cx, sx, gx, K), dw)
+        t += time.perf_counter() - t0
+        del dw
+    out["stack"] = {"us_per_token": 1e6 * t / rows * si.STACK_LAYERS, "unit": "us/token", "cores": cores,
+                    "kind": "oracle", "extrapolated": True,
+                    "sample": f"layer 0 (7 projections) on {rows} token rows, x {si.STACK_LAYERS} layers"}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -519,11 +922,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="vlaq", choices=["vlaq", "reference"])
     ap.add_argument("--ref-rows", type=int, default=4)
-    ap.add_argument("--cpu-rows", type=int, default=768)
+    ap.add_argument("--cpu-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--quick", action="store_true", help="skip the decode / fp8 / e2e extras")
-    ap.add_argument("--stack", action="store_true",
-                    help="also time the 28-layer stack (196 GEMMs) at M = 1024 and M = 1 (about a minute of setup)")
+    ap.add_argument("--quick", action="store_true", help="the prefill step only (no decode / fused / 8-bit / e2e / "
+                                                        "stack sections)")
+    ap.add_argument("--no-stack", action="store_true", help="skip the 28-layer stack (about a minute of setup)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -546,96 +949,18 @@ def main():
     import vlaq_quantize_act_b200 as vq
 
     peaks = load_peaks()
-    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
     # weak scaling: every rank quantizes and multiplies its own tokens (its
     # own activation seeds) against the same weights
     data = make_inputs(M_PREFILL, "cpu", seed_offset=RANK_SEED_STRIDE * rank)
 
-    # ---------------- prefill NVFP4 step (graph replays)
-    step = Step(vq, data, M_PREFILL, device)
-    graph = capture(step)
-    for _ in range(args.warmup):
-        graph.replay()
-    torch.cuda.synchronize()
-    sampler = ClockSampler(local)
-    sampler.start()
-    time.sleep(0.3)
-    ms = time_graph(graph, args.steps, dist_on, device)
-    pro, gem, tmode = kernel_durations(step, max(args.steps // 2, 3))
-    clocks = sampler.stop()
-    value = world * step.flops / (ms / 1e3) / 1e12
-    # dominant kernel: the gate_up GEMM launch (about half of the step)
-    gi = PROJ.index("gate_up")
-    GL = step.layers[gi]
-    gu_ms = statistics.mean(gem[gi])
-    g_ach = 2.0 * M_PREFILL * GL["N"] * GL["K"] / (gu_ms / 1e3) / 1e12
-    gemm_all_ms = sum(statistics.mean(x) for x in gem)
-    gemm_all = step.flops / (gemm_all_ms / 1e3) / 1e12
-    pro_ms = sum(statistics.mean(x) for x in pro)
-    pro_bytes = sum(step.prologue_bytes(L) for L in step.layers)
-    p_ach = pro_bytes / (pro_ms / 1e3) / 1e9
-    per_proj = {L["name"]: {"gemm_us": 1e3 * statistics.mean(gem[i]),
-                            "gemm_tflops": 2.0 * M_PREFILL * L["N"] * L["K"] / (statistics.mean(gem[i]) / 1e3) / 1e12,
-                            "prologue_us": 1e3 * statistics.mean(pro[i]),
-                            "prologue_gbs": step.prologue_bytes(L) / (statistics.mean(pro[i]) / 1e3) / 1e9}
-                for i, L in enumerate(step.layers)}
-    traffic = load_traffic("gemm_nvfp4_prefill")
-
-    out = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "e2m1/e4m3 (fp32 accumulate, bf16 out)", "data": "synthetic",
-        "config": {"workload": "NVFP4 W4A4 prefill: act prologue + block-scaled FP4 GEMM for qkv 3584->4608, "
-                               "o 3584->3584, gate_up 3584->37888, down 18944->3584 (Qwen2.5-VL-7B shapes)",
-                   "global_batch": M_PREFILL * world, "seq_len": M_PREFILL, "parallelism": f"dp{world}",
-                   "l2": "inputs larger than L2 (per-step working set ~294 MB)", "graph": True},
-        "roofline": {"bound": "tensor", "achieved": g_ach, "peak": fp4_peak, "unit": "TFLOP/s",
-                     "frac": g_ach / fp4_peak, "traffic": traffic,
-                     "kernel": "gemm_fp4_sfw_kernel gate_up 1024x37888x3584 (2MNK = 278.1 GFLOP per launch)",
-                     "all_gemms_tflops": gemm_all, "timing": f"CUDA events in a {tmode} capture of the step",
-                     "peak_note": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 4 (nominal FP4:BF16)"},
-        "prologue": {"bound": "hbm", "achieved": p_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": p_ach / peaks["hbm_gbs"], "kernel": "quant_rows_kernel (NVFP4 activation prologue)"},
-        "per_projection": per_proj,
-        "clocks": clocks,
-    }
+    step, out = prefill_section(vq, data, args, dist_on, device, peaks, world)
+    launches_per_step = sum(2 + (1 if L["nb"] else 0) for L in step.layers)
 
     if not args.quick:
-        # ---------------- decode M = 1 (HBM bound), rotating weight copies
-        ddata = {n: (K, N, X[:1].contiguous(), W) for n, (K, N, X, W) in data.items()}
-        dstep = Step(vq, ddata, 1, device, weight_copies=2)
-        dgraph = capture(dstep, copies=2)
-        for _ in range(args.warmup):
-            dgraph.replay()
-        dms = time_graph(dgraph, args.steps, dist_on, device) / 2
-        dbytes = sum(dstep.gemm_bytes(L) + dstep.prologue_bytes(L) for L in dstep.layers)
-        dpro, dgem, _ = kernel_durations(dstep, max(args.steps // 2, 4), copies=2)
-        dgem_ms = sum(sum(x) for x in dgem) / len(dgem[0])
-        dgem_bytes = sum(dstep.gemm_bytes(L) for L in dstep.layers)
-        out["decode"] = {"value": world * dbytes / (dms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": dms,
-                         "bytes_per_step": dbytes, "M": 1,
-                         "gemm_roofline": {"bound": "hbm", "achieved": dgem_bytes / (dgem_ms / 1e3) / 1e9,
-                                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                           "frac": dgem_bytes / (dgem_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
-                         "per_projection_gemm_us": {L["name"]: 1e3 * statistics.mean(dgem[i])
-                                                    for i, L in enumerate(dstep.layers)}}
-        del dstep, dgraph
-
-        # ---------------- FP8 and INT8 W8A8 variants of the prefill step (the
-        # dense 8-bit tensor-core rate is twice bf16 for both kinds)
+        out["decode"] = decode_section(vq, data, args, dist_on, device, peaks, world)
+        out["fused"] = fused_section(vq, data, args, dist_on, device, peaks, world)
         for fmt in ("fp8", "int8"):
-            fstep = Step(vq, data, M_PREFILL, device, fmt=fmt)
-            fgraph = capture(fstep)
-            for _ in range(args.warmup):
-                fgraph.replay()
-            fms = time_graph(fgraph, args.steps, dist_on, device)
-            _, fgem, _ = kernel_durations(fstep, max(args.steps // 2, 3))
-            fgem_ms = sum(sum(x) for x in fgem) / len(fgem[0])
-            fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
-            out[fmt] = {"value": world * fstep.flops / (fms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": fms,
-                        "gemm_achieved": fstep.flops / (fgem_ms / 1e3) / 1e12, "peak": fp8_peak,
-                        "frac": fstep.flops / (fgem_ms / 1e3) / 1e12 / fp8_peak}
-            del fstep, fgraph
+            out[fmt] = w8a8_section(vq, data, args, dist_on, device, peaks, world, fmt)
 
         # ---------------- e2e through the public API with host buffers
         hostX = [L["X"].cpu().pin_memory() for L in step.layers]
@@ -665,12 +990,12 @@ def main():
         out["e2e"] = {"value": world * step.flops / (ems / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ems,
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
-    if not args.quick:
         # ---------------- prologue variants over the four projection inputs:
         # fused RMSNorm + block-64 rotation, per-channel smoothing (divide,
         # before the rotation), both, and a static calibrated global scale
         # (no row-amax pass) plain and fused; same bytes as the plain
         # prologue (the gains and smoothing factors stay in cache)
+        pro_bytes = sum(step.prologue_bytes(L) for L in step.layers)
         variants = {"fused_rmsnorm_wht": (3, False, None), "smooth": (0, True, None),
                     "fused_smooth": (3, True, None), "static": (0, False, 0.01),
                     "fused_static": (3, False, 0.01)}
@@ -728,44 +1053,23 @@ def main():
                                "shape": f"gate_up W {N}x{K} bf16 -> NVFP4 (amax pass + quantize pass)"}
         del wgraph, Wd, wq, ws, wg
 
-    if args.stack:
-        # ---------------- 28-layer stack: one graph of 196 prologue + GEMM pairs
-        # (all NVFP4, then mixed: o / down FP8 W8A8, the rest NVFP4)
-        out["stack"] = {}
-        for prefix, fp8 in (("", ()), ("mixed_", MIXED_FP8)):
-            sw = stack_weights(vq, device, fp8=fp8)
-            for sm in (M_PREFILL, 1):
-                st = Stack(vq, sm, device, weights=sw, fp8=fp8)
-                sg = capture(st)
-                for _ in range(args.warmup):
-                    sg.replay()
-                torch.cuda.synchronize()
-                sms = time_graph(sg, max(args.steps // 4, 3), dist_on, device)
-                key = prefix + ("prefill" if sm > 1 else "decode")
-                out["stack"][key] = {"M": sm, "ms": sms, "us_per_token": 1e3 * sms / sm,
-                                     "tflops": world * st.flops / (sms / 1e3) / 1e12,
-                                     "weight_gbs": world * st.weight_bytes / (sms / 1e3) / 1e9,
-                                     "gemms": len(st.entries), "fp8_projections": list(fp8)}
-                del sg, st
-                torch.cuda.empty_cache()
-            del sw
+        if not args.no_stack:
+            del step
+            torch.cuda.empty_cache()
+            step = None
+            out["stack"] = stack_section(vq, args, dist_on, device, world)
 
-    # launches of our kernels inside the timed region: per step 4 prologues +
-    # 4 GEMMs (+ split-K reductions when planned)
-    launches = sum(2 + (1 if L["nb"] else 0) for L in step.layers) * args.steps
-    out["gpu_launches"] = launches
+    # launches of our kernels inside the headline timed region: per step 4
+    # prologues + 4 GEMMs (+ split-K reductions when planned)
+    out["gpu_launches"] = launches_per_step * args.steps
 
     if rank == 0 and not args.no_cpu_baseline:
-        import oracle
-        t, fl, dec = cpu_oracle_sample(data, 1)
-        t, fl, _ = cpu_oracle_sample(data, args.cpu_rows, decoded_w=dec)
-        out["cpu_baseline"] = {"value": fl / t / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
-                               "kind": "oracle",
-                               "sample": f"{args.cpu_rows} token rows of each projection: NVFP4 quantize + fp64 "
-                                         f"GEMM ({t:.1f} s)"}
+        base = cpu_baselines(data, args)
+        out["cpu_baseline"] = dict(base["prefill"])
+        out["cpu_baseline"]["cpu"] = base["cpu"]
+        out["cpu_baseline"]["workloads"] = {k: v for k, v in base.items() if k not in ("prefill", "cores", "cpu")}
     if rank == 0:
         print(json.dumps(out), flush=True)
-    del graph
     if dist_on:
         torch.distributed.destroy_process_group()
 
