@@ -551,6 +551,9 @@ def run_reference(args, rank):
     print(json.dumps(out), flush=True)
 
 
+SECTIONS = ("decode", "fused", "w8a8", "e2e", "variants", "weight_quant", "stack")
+
+
 class Launches:
     """run() issues the given launches in order (a graph of them is timed
     back to back)."""
@@ -927,8 +930,16 @@ def main():
     ap.add_argument("--quick", action="store_true", help="the prefill step only (no decode / fused / 8-bit / e2e / "
                                                         "stack sections)")
     ap.add_argument("--no-stack", action="store_true", help="skip the 28-layer stack (about a minute of setup)")
+    ap.add_argument("--sections", default=",".join(SECTIONS),
+                    help="comma-separated sections to run after the prefill step: " + ", ".join(SECTIONS))
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    sections = set() if args.quick else {x for x in args.sections.split(",") if x}
+    if args.no_stack:
+        sections.discard("stack")
+    unknown = sections - set(SECTIONS)
+    if unknown:
+        ap.error(f"unknown sections {sorted(unknown)}")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -956,12 +967,14 @@ def main():
     step, out = prefill_section(vq, data, args, dist_on, device, peaks, world)
     launches_per_step = sum(2 + (1 if L["nb"] else 0) for L in step.layers)
 
-    if not args.quick:
+    if "decode" in sections:
         out["decode"] = decode_section(vq, data, args, dist_on, device, peaks, world)
+    if "fused" in sections:
         out["fused"] = fused_section(vq, data, args, dist_on, device, peaks, world)
+    if "w8a8" in sections:
         for fmt in ("fp8", "int8"):
             out[fmt] = w8a8_section(vq, data, args, dist_on, device, peaks, world, fmt)
-
+    if "e2e" in sections:
         # ---------------- e2e through the public API with host buffers
         hostX = [L["X"].cpu().pin_memory() for L in step.layers]
         hostY = [torch.empty(L["Y"].shape, dtype=torch.bfloat16).pin_memory() for L in step.layers]
@@ -990,6 +1003,7 @@ def main():
         out["e2e"] = {"value": world * step.flops / (ems / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ems,
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    if "variants" in sections:
         # ---------------- prologue variants over the four projection inputs:
         # fused RMSNorm + block-64 rotation, per-channel smoothing (divide,
         # before the rotation), both, and a static calibrated global scale
@@ -1031,6 +1045,7 @@ def main():
                                                "frac": pro_bytes / (pms / 1e3) / 1e9 / peaks["hbm_gbs"]}
             del pgraph
 
+    if "weight_quant" in sections:
         # ---------------- offline weight quantization (a1), gate_up weights:
         # HBM-bound; algorithmic bytes = one bf16 read + codes, scales, g
         K, N, _, W = data["gate_up"]
@@ -1053,11 +1068,11 @@ def main():
                                "shape": f"gate_up W {N}x{K} bf16 -> NVFP4 (amax pass + quantize pass)"}
         del wgraph, Wd, wq, ws, wg
 
-        if not args.no_stack:
-            del step
-            torch.cuda.empty_cache()
-            step = None
-            out["stack"] = stack_section(vq, args, dist_on, device, world)
+    if "stack" in sections:
+        del step
+        torch.cuda.empty_cache()
+        step = None
+        out["stack"] = stack_section(vq, args, dist_on, device, world)
 
     # launches of our kernels inside the headline timed region: per step 4
     # prologues + 4 GEMMs (+ split-K reductions when planned)
