@@ -202,13 +202,14 @@ def test_split_workspace_reused_across_calls_and_shapes():
 
 
 # one or two token rows against weights of at most 2^25 elements take the
-# weight-streaming CUDA-core kernel (larger M or weights the tensor-core one):
-# ragged K (K % 64 in {16, 32, 48}, K = 16), N = 8, a partial last group of
-# rows per CTA, the decode projection shapes, residual on and off
+# weight-streaming CUDA-core kernel (larger M or weights the tensor-core
+# one, split K): ragged K (K % 64 in {16, 32, 48}, K = 16), N = 8, a partial
+# last group of rows per CTA, the decode projection shapes, up to 32 token
+# rows, residual on and off
 FEW_ROW_CASES = [(1, 8, 16, False), (2, 24, 48, True), (3, 136, 208, False), (4, 512, 4096, True),
                  (1, 4608, 3584, True), (4, 4608, 3584, False), (1, 3584, 18944, True), (2, 3584, 18944, False),
-                 (3, 40, 336, True), (1, 37888, 3584, False),
-                 (2, 1024, 18944, True)]  # the few-row kernel with more than 48 KB of shared memory
+                 (3, 40, 336, True), (1, 37888, 3584, False), (8, 37888, 3584, True), (32, 1000, 1024, True),
+                 (17, 3584, 18944, False), (2, 1024, 18944, True)]
 
 
 @pytest.mark.parametrize("M,N,K,res", FEW_ROW_CASES + [(2, 4608, 3584, True), (2, 3584, 3584, False)])
@@ -226,10 +227,10 @@ def test_linear_nvfp4_few_rows(M, N, K, res):
            to_dev(layouts.pad_codes(cw, K)), to_dev(layouts.tile_scales(sw, N, K)), to_dev(gw))
     Y = gpu_linear_nvfp4(*dev, M, N, K, None if R is None else R.cuda())
     check_gemm(Y, Y64, dx, dw, K, residual_f64(R), f"few rows M={M} N={N} K={K} res={res}")
-    # the CUDA-core kernel needs no workspace; a second call gives the same bits
-    few = M <= 2 and N * K <= 1 << 25
+    # a second call gives the same bits (a shape without a split plan runs
+    # without a workspace)
     Y2 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
-    wsp, nb = (None, 0) if few else m.alloc_workspace(M, N, K)
+    wsp, nb = (None, 0) if m.vlaq_linear_workspace_bytes(M, N, K) == 0 else m.alloc_workspace(M, N, K)
     m.vlaq_linear_nvfp4(*dev, None if R is None else R.cuda(), Y2, M, N, K, wsp, nb)
     torch.cuda.synchronize()
     m.vlaq_check()

@@ -255,27 +255,6 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   return out;
 }
 
-// Markstein's correction step (see markstein_quotient in quant.cu) on two
-// values at once with the packed fp32x2 instructions of sm_100a (each lane
-// rounded once, subnormals kept):  q0 = x y, e = q0 S - x (x negated by a
-// multiply by -1, exact), q = q0 + e (-y).  Bit-identical to the scalar
-// form, zeros' signs included.
-__device__ __forceinline__ void markstein_pair(float x0, float x1, float S, float y, float& q0out, float& q1out) {
-  asm("{\n\t.reg .b64 x, y, ny, s, m1, q0, nx, e, q;\n\t"
-      "mov.b64 x, {%2, %3};\n\t"
-      "mov.b64 y, {%4, %4};\n\t"
-      "mov.b64 ny, {%5, %5};\n\t"
-      "mov.b64 s, {%6, %6};\n\t"
-      "mov.b64 m1, {%7, %7};\n\t"
-      "mul.rn.f32x2 q0, x, y;\n\t"
-      "mul.rn.f32x2 nx, x, m1;\n\t"
-      "fma.rn.f32x2 e, q0, s, nx;\n\t"
-      "fma.rn.f32x2 q, e, ny, q0;\n\t"
-      "mov.b64 {%0, %1}, q;\n\t}"
-      : "=f"(q0out), "=f"(q1out)
-      : "f"(x0), "f"(x1), "f"(y), "f"(-y), "f"(S), "f"(-1.0f));
-}
-
 // One E4M3 byte -> fp32 (exact).
 __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
   uint32_t h2;

@@ -1,21 +1,23 @@
 // Fused activation prologue and the offline weight quantizers.
 //
-// Persistent CTAs, several per SM, each keeping up to four rows in flight in
-// a shared-memory ring: thread 0 fetches a whole bf16 row with one bulk copy
-// (cp.async.bulk, completion on the slot's mbarrier) and the CTA quantizes
-// the oldest staged row while the next ones stream in, so HBM sees a steady
-// queue of large reads instead of one dependent load-reduce-store chain per
-// row.  A staged row is read twice from shared memory:
-//   pass A  (transform and) per-16 block amax, kept in registers; row amax
-//           -> global scale g of the row;
-//   pass B  transform again, E4M3 block scale, codes.
-// Lane l of warp w owns the 16-element block 32 (W it + w) + l of the row (W
-// warps per CTA): one NVFP4 scale byte and 8 code bytes, so four lanes hold
-// one Hadamard block and one 4-byte word of the 128x4 tiled scale layout,
-// and a warp writes 256 (NVFP4) or 512 (FP8) contiguous code bytes per step.
-// HBM-bound: 2 bytes in and 0.5625 (NVFP4) or 1 (FP8) bytes out per element.
-// Short rows (K <= 8192) run 8-warp CTAs, four per SM; long rows 16-warp
-// CTAs, two per SM, so one row is spread over more lanes.
+// Rows are held in registers.  A CTA of W warps owns one row at a time (4
+// warps for rows of up to 4096 elements, 8 for longer rows); lane l of warp
+// w holds the 16-element blocks 32 (W i + w) + l of the row, i = 0 .. BPL-1
+// (2 blocks per lane for short rows, 5 or 8 for long ones), read with two
+// coalesced 16-byte loads each (a warp reads 1 KiB of contiguous bf16 per
+// block index).  Per row:
+//   pass A  (transform and) per-16 block amax; the transformed values of
+//           the fused variants (RMSNorm, rotation, smoothing) are kept in
+//           shared memory so each is computed once; row amax by one warp
+//           reduction and a cross-warp max -> global scale g;
+//   pass B  E4M3 block scale and codes from the kept values (or the bf16
+//           words still in registers), stored with coalesced 8- or 16-byte
+//           stores.
+// Four lanes hold one Hadamard block (stages h = 1, 2, 4, 8 inside a lane,
+// 16 and 32 across lanes) and one 4-byte word of the 128x4 tiled scale
+// layout; a warp writes 256 (NVFP4) or 512 (FP8, INT8) contiguous code
+// bytes per block index.  HBM-bound: 2 bytes in and 0.5625 (NVFP4) or 1
+// (FP8, INT8) bytes out per element.
 //
 // Arithmetic follows the format definitions stated in include/vlaq.h: every
 // fp32 operation is an explicitly rounded intrinsic (no contraction),
@@ -44,17 +46,17 @@ namespace {
 enum { kNvfp4 = 0, kFp8 = 1, kInt8 = 2 };
 enum { kPerRow = 0, kTensorAmax = 1, kTensorQuant = 2, kStatic = 3 };
 
-constexpr int kMaxRowBufs = 4;
-constexpr int kMidRowK = 4096;    // many rows up to this length: 4-warp CTAs, 8 per SM
-constexpr int kShortRowK = 8192;  // rows up to this length take the 8-warp CTAs
-
-// CTA shape per row length: W warps, CTAs resident per SM, ring budget.
-template <int W>
+// Row-group shape: W warps per row, at most BPL 16-element blocks per lane
+// (8 bf16 words each, kept in registers).
+template <int W, int BPL>
 struct RowCfg {
-  static constexpr int kThreads = 32 * W;
-  static constexpr int kCtasPerSm = 1024 / kThreads;  // 32 warps per SM, 64 registers a thread
-  static constexpr int kRingBytes = (W == 4) ? 26 * 1024 : (W == 8) ? 52 * 1024 : 110 * 1024;
-  static constexpr int kMaxK = (W == 4) ? kMidRowK : (W == 8) ? kShortRowK : int(kMaxQuantK);
+  static_assert(W >= 2, "a row group is a whole CTA");
+  static constexpr int kMaxK = 16 * 32 * W * BPL;
+  static constexpr int kWarps = W;  // warps per CTA (one row group)
+  static constexpr int kThreads = 32 * kWarps;
+  // kept transformed values of the fused variants: per warp BPL x 16 fp32
+  // per lane
+  static constexpr int kCacheBytesPerWarp = BPL * 16 * 4 * 32;
 };
 
 __device__ __forceinline__ void unpack_bf16x8(const uint4& q, float* v) {
@@ -115,14 +117,38 @@ __device__ __forceinline__ float markstein_quotient(float x, float S, float y) {
 template <int N>
 __device__ __forceinline__ void quotients(const float* v, const Divisor& d, float* q) {
   static_assert(N % 2 == 0, "pairs");
+  // the same three steps on packed pairs (sm_100a fp32x2 multiply and fused
+  // multiply-add, each lane rounded once): q0 = x y, e = q0 S - x (x negated
+  // exactly, so -0 stays -0), q = q0 + e (-y)
+  const float2 yy = make_float2(d.y, d.y);
+  const float2 ny = make_float2(-d.y, -d.y);
+  const float2 ss = make_float2(d.S, d.S);
 #pragma unroll
-  for (int i = 0; i < N; i += 2) markstein_pair(v[i], v[i + 1], d.S, d.y, q[i], q[i + 1]);
+  for (int i = 0; i < N; i += 2) {
+    const float2 x = make_float2(v[i], v[i + 1]);
+    const float2 q0 = __fmul2_rn(x, yy);
+    const float2 e = __ffma2_rn(q0, ss, make_float2(-x.x, -x.y));
+    const float2 r = __ffma2_rn(e, ny, q0);
+    q[i] = r.x;
+    q[i + 1] = r.y;
+  }
   if (__any_sync(0xffffffffu, d.slow)) {
     if (d.slow) {
 #pragma unroll
       for (int i = 0; i < N; ++i) q[i] = (d.S == 0.0f) ? 0.0f : __fdiv_rn(v[i], d.S);
     }
   }
+}
+
+// The global scale of a row from its amax A >= 0: RN(A / 2688) (NVFP4),
+// RN(A / 448) (FP8) or RN(A / 127) (INT8), by the correction step against
+// the constant's correctly rounded reciprocal; rows whose amax is tiny
+// (quotient near the subnormal range) take a divide.  Uniform per row.
+template <int FMT>
+__device__ __forceinline__ float row_global(float A) {
+  constexpr float c = (FMT == 0) ? 2688.0f : (FMT == 1) ? 448.0f : 127.0f;
+  if (A < 0x1p-64f) return __fdiv_rn(A, c);
+  return markstein_quotient(A, c, __frcp_rn(c));
 }
 
 // E4M3 byte of RN(a / d) for a >= 0 (d is warp-uniform).
@@ -151,9 +177,6 @@ struct RowArgs {
   const float* smooth;  // per-input-channel smoothing factors [K] (or null)
   uint32_t sflags;      // kFlagSmoothAfter | kFlagSmoothMul
   float g_static;       // calibrated global scale (kStatic)
-  int nbuf;       // ring depth (rows in flight per CTA)
-  int row_bytes;  // ring slot size (2 K rounded up to 128)
-  long long budget;
 };
 
 // Normalised WHT of the 64-block spread over lanes 4 g .. 4 g + 3 (16 values
@@ -200,14 +223,14 @@ __device__ __forceinline__ void smooth_block(const RowArgs& a, int q, float* v) 
 
 // The 16 values of block q after the row transform (zeros past the row):
 // y = (x r) gamma for RMSNorm, the smoothing divide (or multiply) before or
-// after the block-64 WHT.  Warp-uniform.
+// after the block-64 WHT.  x is the block's two bf16 words (zero past the
+// row).  Warp-uniform.
 template <bool NORM, bool WHT, bool SMOOTH>
-__device__ __forceinline__ void block_values(const RowArgs& a, const uint8_t* rs, int q, int nblk16, float r,
-                                             int lane, float* v) {
+__device__ __forceinline__ void block_values(const RowArgs& a, const uint4& x0, const uint4& x1, int q, int nblk16,
+                                             float r, int lane, float* v) {
+  unpack_bf16x8(x0, v);
+  unpack_bf16x8(x1, v + 8);
   if (q < nblk16) {
-    const uint4* src = reinterpret_cast<const uint4*>(rs) + 2 * q;
-    unpack_bf16x8(src[0], v);
-    unpack_bf16x8(src[1], v + 8);
     if (NORM) {
       const uint4* gsrc = reinterpret_cast<const uint4*>(a.gamma) + 2 * q;
       float gm[16];
@@ -217,9 +240,6 @@ __device__ __forceinline__ void block_values(const RowArgs& a, const uint8_t* rs
       for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(__fmul_rn(v[j], r), gm[j]);
     }
     if (SMOOTH && !(a.sflags & kFlagSmoothAfter)) smooth_block(a, q, v);
-  } else {
-#pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = 0.0f;
   }
   if (WHT) wht64_lanes(v, lane);
   if (SMOOTH && (a.sflags & kFlagSmoothAfter) && q < nblk16) smooth_block(a, q, v);
@@ -232,131 +252,135 @@ __device__ __forceinline__ float absmax16(const float* v) {
   return m;
 }
 
-// All rows of one launch: FMT (NVFP4 / FP8), MODE (per-row scale, tensor
-// amax pass, tensor quantize pass, static calibrated scale), NORM (RMSNorm,
-// per-row and static modes), WHT (block-64 Hadamard), W warps per CTA.  Persistent grid: the CTA takes rows
-// blockIdx.x + i gridDim.x, the ring slot of row i is i mod nbuf.
-template <int FMT, int MODE, bool NORM, bool WHT, bool SMOOTH, int W>
-__global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) quant_rows_kernel(const RowArgs a) {
-  constexpr int T = RowCfg<W>::kThreads;
-  constexpr int MAXIT = RowCfg<W>::kMaxK / 16 / T;  // blocks per lane, at most
-  extern __shared__ __align__(128) uint8_t s_ring[];
-  __shared__ __align__(8) uint64_t s_bar[kMaxRowBufs];
-  __shared__ float s_red[W];
+// RMSNorm factor r = 1 / sqrt(mean(x^2) + eps) of a row: the warps put their
+// blocks into a shared-memory copy of the row, and one warp walks it in the
+// fixed tree's order (lane l: the 8-element chunks l, l + 32, ..., the
+// chain's next chunk loaded before the current chunk's eight steps; then
+// the XOR butterfly).
+__device__ __forceinline__ float rms_factor_row(const uint4* x4, int K, float eps, int lane) {
+  const int nch = K >> 3;
+  float acc = 0.0f;
+  uint4 cur = lane < nch ? x4[lane] : make_uint4(0, 0, 0, 0);
+  for (int c = lane; c < nch; c += 32) {
+    const uint4 nxt = c + 32 < nch ? x4[c + 32] : make_uint4(0, 0, 0, 0);
+    float t[8];
+    unpack_bf16x8(cur, t);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc = __fmaf_rn(t[j], t[j], acc);
+    cur = nxt;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
+  const float mean = __fdiv_rn(acc, static_cast<float>(K));
+  return __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean, eps)));
+}
+
+// All rows of one launch: FMT (NVFP4 / FP8 / INT8), MODE (per-row scale,
+// tensor amax pass, tensor quantize pass, static calibrated scale), NORM
+// (RMSNorm, per-row and static modes), WHT (block-64 Hadamard), SMOOTH
+// (per-channel smoothing), W warps per row.  Row group k of the grid takes
+// rows k, k + groups, ... (one row per group at the workload sizes).
+template <int FMT, int MODE, bool NORM, bool WHT, bool SMOOTH, int W, int BPL>
+__global__ void __launch_bounds__(RowCfg<W, BPL>::kThreads) quant_rows_kernel(const RowArgs a) {
+  using C = RowCfg<W, BPL>;
+  constexpr bool KEEP = NORM || WHT || SMOOTH;  // transformed values kept in shared memory
+  // dynamic shared memory: [kept values][row copy]
+  extern __shared__ __align__(16) float4 s_keep[];
+  __shared__ float s_red[C::kWarps];
   __shared__ float s_r;
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wr = warp;  // warp index inside the row group
   const int K = a.K;
   const int nblk16 = K >> 4;
   const int nblk64 = (K + 63) >> 6;
   const int nblk16_pad = 4 * nblk64;  // blocks up to the padded row end
-  const int iters = (nblk16_pad + T - 1) / T;
-  const int nbuf = a.nbuf;
-  const uint32_t row_tx = static_cast<uint32_t>(2 * K);
-  const int64_t stride = gridDim.x;
+  const int64_t gstride = gridDim.x;
+  float4* keep = s_keep + static_cast<size_t>(warp) * BPL * 4 * 32;
 
-  if (tid == 0) {
-    for (int b = 0; b < nbuf; ++b) mbar_init(&s_bar[b], 1);
-    fence_mbarrier_init();
-  }
-  __syncthreads();
   griddep_wait();
   griddep_launch_dependents();
 
-  if (tid == 0) {
-    for (int b = 0; b < nbuf; ++b) {
-      const int64_t row = blockIdx.x + b * stride;
-      if (row >= a.rows) break;
-      mbar_arrive_expect_tx(&s_bar[b], row_tx);
-      bulk_load(s_ring + b * a.row_bytes, a.X + row * K, row_tx, &s_bar[b]);
-    }
-  }
   float g_tensor = 0.0f;
   if (MODE == kTensorQuant) g_tensor = __fdiv_rn(__uint_as_float(*a.amax_word), 2688.0f);
   if (MODE == kStatic) g_tensor = a.g_static;
 
-  int slot = 0;
-  uint32_t phase = 0;
-  for (int64_t row = blockIdx.x; row < a.rows; row += stride) {
-    const bool ok = __syncthreads_and(mbar_wait(&s_bar[slot], phase, a.budget));
-    if (!ok) {
-      // record it, let the copies still in flight land, and stop
-      if (tid == 0) {
-        atomicOr(&g_vlaq_quant_status, kStatusTimeout);
-        for (int k = 0; k < nbuf && row + k * stride < a.rows; ++k) {
-          const int sk = slot + k;
-          mbar_wait(&s_bar[sk % nbuf], phase ^ (sk >= nbuf ? 1u : 0u), a.budget);
-        }
+  for (int64_t row = blockIdx.x; row < a.rows; row += gstride) {
+    // ---- the row's blocks into registers (zero past the row end)
+    const uint4* x4 = reinterpret_cast<const uint4*>(a.X + row * K);
+    uint4 d[BPL][2];
+#pragma unroll
+    for (int i = 0; i < BPL; ++i) {
+      const int q = (i * W + wr) * 32 + lane;
+      if (q < nblk16) {
+        d[i][0] = __ldg(x4 + 2 * q);
+        d[i][1] = __ldg(x4 + 2 * q + 1);
+      } else {
+        d[i][0] = make_uint4(0, 0, 0, 0);
+        d[i][1] = make_uint4(0, 0, 0, 0);
       }
-      break;
     }
-    const uint8_t* rs = s_ring + slot * a.row_bytes;
 
-    // ---- RMSNorm factor r = 1 / sqrt(mean(x^2) + eps), fixed 32-lane tree
+    // ---- RMSNorm factor, fixed 32-lane tree
     float r = 1.0f;
     if (NORM) {
-      if (warp == 0) {
-        // the chain of fused multiply-adds is fixed; the next chunk's load
-        // is issued before the current chunk's eight steps
-        const uint4* rs4 = reinterpret_cast<const uint4*>(rs);
-        const int nch = K >> 3;
-        float acc = 0.0f;
-        uint4 cur = lane < nch ? rs4[lane] : make_uint4(0, 0, 0, 0);
-        for (int c = lane; c < nch; c += 32) {
-          const uint4 nxt = c + 32 < nch ? rs4[c + 32] : make_uint4(0, 0, 0, 0);
-          float t[8];
-          unpack_bf16x8(cur, t);
+      // the row's copy follows the kept values in shared memory
+      uint4* srow4 = reinterpret_cast<uint4*>(s_keep + static_cast<size_t>(C::kWarps) * BPL * 4 * 32);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc = __fmaf_rn(t[j], t[j], acc);
-          cur = nxt;
+      for (int i = 0; i < BPL; ++i) {
+        const int q = (i * W + wr) * 32 + lane;
+        if (q < nblk16) {
+          srow4[2 * q] = d[i][0];
+          srow4[2 * q + 1] = d[i][1];
         }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
-        if (lane == 0) {
-          const float mean = __fdiv_rn(acc, static_cast<float>(K));
-          s_r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean, a.eps)));
-        }
+      }
+      __syncthreads();
+      if (wr == 0) {
+        const float rr = rms_factor_row(srow4, K, a.eps, lane);
+        if (lane == 0) s_r = rr;
       }
       __syncthreads();
       r = s_r;
     }
 
-    // ---- pass A: per-block amax (kept in registers) and row amax
-    float a16r[MAXIT];
-    float g = g_tensor;
-    if (MODE == kStatic && tid == 0) a.gout[row] = g;
-    if (MODE == kPerRow || MODE == kTensorAmax) {
-      float local = 0.0f;
+    // ---- pass A: per-block amax (kept in registers), transformed values
+    // kept in shared memory, row amax
+    float a16r[BPL];
+    float local = 0.0f;
 #pragma unroll
-      for (int it = 0; it < MAXIT; ++it) {
-        a16r[it] = 0.0f;
-        if (it < iters && (it * W + warp) * 32 < nblk16_pad) {
-          const int q = (it * W + warp) * 32 + lane;
-          float m = 0.0f;
-          if (NORM || WHT || SMOOTH) {
-            float v[16];
-            block_values<NORM, WHT, SMOOTH>(a, rs, q, nblk16, r, lane, v);
-            m = absmax16(v);
-          } else if (q < nblk16) {
-            const uint4* src = reinterpret_cast<const uint4*>(rs) + 2 * q;
-            m = absmax_bf16x16(src[0], src[1]);
-          }
-          a16r[it] = m;
-          local = fmaxf(local, m);
+    for (int i = 0; i < BPL; ++i) {
+      a16r[i] = 0.0f;
+      if ((i * W + wr) * 32 < nblk16_pad) {  // warp-uniform
+        const int q = (i * W + wr) * 32 + lane;
+        float m;
+        if (KEEP) {
+          float v[16];
+          block_values<NORM, WHT, SMOOTH>(a, d[i][0], d[i][1], q, nblk16, r, lane, v);
+          m = absmax16(v);
+#pragma unroll
+          for (int t = 0; t < 4; ++t)
+            keep[(i * 4 + t) * 32 + lane] = make_float4(v[4 * t], v[4 * t + 1], v[4 * t + 2], v[4 * t + 3]);
+        } else {
+          m = absmax_bf16x16(d[i][0], d[i][1]);
         }
+        a16r[i] = m;
+        local = fmaxf(local, m);
       }
+    }
+    float g = g_tensor;
+    if (MODE == kStatic && wr == 0 && lane == 0) a.gout[row] = g;
+    if (MODE == kPerRow || MODE == kTensorAmax) {
       // non-negative floats order like their bit patterns: one warp reduction
-      local = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(local)));
-      if (lane == 0) s_red[warp] = local;
+      float A = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(local)));
+      if (lane == 0) s_red[wr] = A;
       __syncthreads();
-      float A = s_red[0];
+      A = s_red[0];
 #pragma unroll
       for (int w = 1; w < W; ++w) A = fmaxf(A, s_red[w]);
       if (MODE == kTensorAmax) {
-        if (tid == 0) atomicMax(a.amax_word, __float_as_uint(A));  // A >= 0: bit order = value order
+        if (wr == 0 && lane == 0) atomicMax(a.amax_word, __float_as_uint(A));  // A >= 0: bit order = value order
       } else {
-        g = (FMT == kNvfp4) ? __fdiv_rn(A, 2688.0f) : __fdiv_rn(A, FMT == kFp8 ? 448.0f : 127.0f);
-        if (tid == 0) a.gout[row] = g;
+        g = row_global<FMT>(A);
+        if (wr == 0 && lane == 0) a.gout[row] = g;
       }
     }
 
@@ -367,12 +391,24 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
         uint8_t* srow = a.scales + scale_row_base(row, nblk64);
         const Divisor d6g = make_divisor(__fmul_rn(6.0f, g));
 #pragma unroll
-        for (int it = 0; it < MAXIT; ++it) {
-          if (it < iters && (it * W + warp) * 32 < nblk16_pad) {
-            const int q = (it * W + warp) * 32 + lane;
+        for (int i = 0; i < BPL; ++i) {
+          if ((i * W + wr) * 32 < nblk16_pad) {
+            const int q = (i * W + wr) * 32 + lane;
             float v[16];
-            block_values<NORM, WHT, SMOOTH>(a, rs, q, nblk16, r, lane, v);
-            float a16 = (MODE == kPerRow) ? a16r[it] : absmax16(v);
+            if (KEEP) {
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                const float4 f = keep[(i * 4 + t) * 32 + lane];
+                v[4 * t] = f.x;
+                v[4 * t + 1] = f.y;
+                v[4 * t + 2] = f.z;
+                v[4 * t + 3] = f.w;
+              }
+            } else {
+              unpack_bf16x8(d[i][0], v);
+              unpack_bf16x8(d[i][1], v + 8);
+            }
+            float a16 = a16r[i];
             uint32_t sb8 = 0;
             float S = 0.0f;
             if (g > 0.0f) {
@@ -403,11 +439,23 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
       } else {
         const Divisor dg = make_divisor(g);
 #pragma unroll
-        for (int it = 0; it < MAXIT; ++it) {
-          if (it < iters && (it * W + warp) * 32 < nblk16_pad) {
-            const int q = (it * W + warp) * 32 + lane;
+        for (int i = 0; i < BPL; ++i) {
+          if ((i * W + wr) * 32 < nblk16_pad) {
+            const int q = (i * W + wr) * 32 + lane;
             float v[16];
-            block_values<NORM, WHT, SMOOTH>(a, rs, q, nblk16, r, lane, v);
+            if (KEEP) {
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                const float4 f = keep[(i * 4 + t) * 32 + lane];
+                v[4 * t] = f.x;
+                v[4 * t + 1] = f.y;
+                v[4 * t + 2] = f.z;
+                v[4 * t + 3] = f.w;
+              }
+            } else {
+              unpack_bf16x8(d[i][0], v);
+              unpack_bf16x8(d[i][1], v + 8);
+            }
             float qv[16];
             quotients<16>(v, dg, qv);
             uint32_t w[4];
@@ -433,21 +481,8 @@ __global__ void __launch_bounds__(RowCfg<W>::kThreads, RowCfg<W>::kCtasPerSm) qu
         }
       }
     }
-
-    // ---- every thread is done with this slot: refill it with the row nbuf steps ahead
+    // the next row reuses s_red / s_r
     __syncthreads();
-    if (tid == 0) {
-      const int64_t next = row + nbuf * stride;
-      if (next < a.rows) {
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&s_bar[slot], row_tx);
-        bulk_load(s_ring + slot * a.row_bytes, a.X + next * K, row_tx, &s_bar[slot]);
-      }
-    }
-    if (++slot == nbuf) {
-      slot = 0;
-      phase ^= 1u;
-    }
   }
 }
 
@@ -457,34 +492,36 @@ __global__ void finalize_global_kernel(float* g) {
   g[0] = __fdiv_rn(__uint_as_float(*reinterpret_cast<unsigned int*>(g)), 2688.0f);
 }
 
-template <int FMT, int MODE, bool NORM, bool WHT, bool SMOOTH, int W>
-cudaError_t launch_ring(RowArgs a, cudaStream_t s) {
-  using C = RowCfg<W>;
-  auto kern = quant_rows_kernel<FMT, MODE, NORM, WHT, SMOOTH, W>;
-  const int fit = C::kRingBytes / a.row_bytes;
-  a.nbuf = fit < 2 ? 2 : (fit > kMaxRowBufs ? kMaxRowBufs : fit);  // 2 x 64 KiB at the largest K
-  const size_t smem = static_cast<size_t>(a.nbuf) * a.row_bytes;
+template <int FMT, int MODE, bool NORM, bool WHT, bool SMOOTH, int W, int BPL>
+cudaError_t launch_groups(const RowArgs& a, cudaStream_t s) {
+  using C = RowCfg<W, BPL>;
+  auto kern = quant_rows_kernel<FMT, MODE, NORM, WHT, SMOOTH, W, BPL>;
+  const bool keep = NORM || WHT || SMOOTH;
+  size_t smem = keep ? static_cast<size_t>(C::kWarps) * C::kCacheBytesPerWarp : 0;
+  if (NORM) smem += static_cast<size_t>(2) * a.K;  // the row's copy for the tree
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  // resident CTAs per SM: the register limit, or fewer where the rings do
-  // not fit (1 KiB per CTA is reserved by the SM)
-  int per_sm = static_cast<int>(228 * 1024 / (smem + 2048));
-  per_sm = per_sm < 1 ? 1 : (per_sm > C::kCtasPerSm ? C::kCtasPerSm : per_sm);
-  const int64_t ctas = static_cast<int64_t>(device_sm_count()) * per_sm;
-  const unsigned int grid = static_cast<unsigned int>(a.rows < ctas ? a.rows : ctas);
+  // one row per CTA while rows last; very tall inputs loop (at most 64
+  // CTAs per SM are launched)
+  const int64_t ctas = a.rows;
+  const int64_t cap = static_cast<int64_t>(device_sm_count()) * 64;
+  const unsigned int grid = static_cast<unsigned int>(ctas < cap ? ctas : cap);
   return launch_pdl(kern, dim3(grid), dim3(C::kThreads), smem, s, a);
 }
 
 template <int FMT, int MODE, bool NORM, bool WHT, bool SMOOTH = false>
 cudaError_t launch_shape(const RowArgs& a, cudaStream_t s) {
-  // short rows and enough of them for every SM: one row per small CTA, so
-  // more rows are worked on at once; few rows keep the 8-warp CTAs (shorter
-  // per-row chains)
-  if (a.K <= kMidRowK && a.rows >= 2 * device_sm_count()) return launch_ring<FMT, MODE, NORM, WHT, SMOOTH, 4>(a, s);
-  if (a.K <= kShortRowK) return launch_ring<FMT, MODE, NORM, WHT, SMOOTH, 8>(a, s);
-  return launch_ring<FMT, MODE, NORM, WHT, SMOOTH, 16>(a, s);
+  // measured on B200 (graph-timed launches over inputs larger than L2,
+  // M = 1024): rows of up to 4096 elements run fastest with 4 warps per row
+  // and 2 blocks per lane (against 1, 2 or 8 warps), rows of up to 20480
+  // with 8 warps and 5 blocks per lane (against 4 or 16 warps); loading the
+  // rows into registers beat staging them through a shared-memory ring of
+  // bulk copies at both lengths
+  if (a.K <= RowCfg<4, 2>::kMaxK) return launch_groups<FMT, MODE, NORM, WHT, SMOOTH, 4, 2>(a, s);
+  if (a.K <= RowCfg<8, 5>::kMaxK) return launch_groups<FMT, MODE, NORM, WHT, SMOOTH, 8, 5>(a, s);
+  return launch_groups<FMT, MODE, NORM, WHT, SMOOTH, 8, 8>(a, s);
 }
 
 template <int FMT, int MODE>
@@ -505,9 +542,6 @@ cudaError_t launch_rows(const void* X, int64_t rows, int64_t K, const void* gamm
   a.smooth = smooth;
   a.sflags = flags & (kFlagSmoothAfter | kFlagSmoothMul);
   a.g_static = g_static;
-  a.nbuf = 0;
-  a.row_bytes = static_cast<int>((2 * K + 127) / 128 * 128);
-  a.budget = kWaitBudgetCycles;
   const bool wht = (flags & kFlagHadamard) != 0;
   if constexpr ((MODE == kPerRow || MODE == kStatic) && FMT == kNvfp4) {
     if (smooth) {
