@@ -501,18 +501,21 @@ struct SfwCfg {
   static constexpr int B_BYTES = BN * 128;
   static constexpr int SFA_BYTES = 4 * 512;
   static constexpr int SFB_BYTES = NRB * 4 * 512;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int STAGES = (220 * 1024) / STAGE_BYTES;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // operand tiles of one stage
+  static constexpr int STAGES = 4;
+  static constexpr int SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;  // scale atoms of one stage
+  static constexpr int SF_STAGES = 4;
   static constexpr int NSF = 4;                       // TMEM scale buffers
   static constexpr int SF_COLS = 16 + 16 * NRB;        // per buffer: 16 (A) + 32 (B)
   static constexpr int SF_COL0 = BN;                   // after the accumulator
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SF_STAGES * SF_STAGE_BYTES + 1024;
   static constexpr int THREADS = 512;
   static constexpr int EPI_WARPS = 8;
   static constexpr uint32_t IDESC =
       (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
   static_assert(SF_COL0 + NSF * SF_COLS <= kTmemCols, "TMEM budget");
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
 __global__ void __launch_bounds__(SfwCfg::THREADS, 1)
@@ -524,6 +527,8 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
   __shared__ __align__(8) uint64_t sff_bar[C::NSF];
   __shared__ __align__(8) uint64_t sfe_bar[C::NSF];
+  __shared__ __align__(8) uint64_t sfsf_bar[C::SF_STAGES];  // scale atoms landed
+  __shared__ __align__(8) uint64_t sfse_bar[C::SF_STAGES];  // scale atoms copied to TMEM
   __shared__ __align__(8) uint64_t accf_bar;
   __shared__ __align__(8) uint64_t acce_bar;
   __shared__ __align__(8) uint64_t drain_bar;
@@ -545,6 +550,10 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       mbar_init(&sff_bar[i], 4);
       mbar_init(&sfe_bar[i], 1);
     }
+    for (int i = 0; i < C::SF_STAGES; ++i) {
+      mbar_init(&sfsf_bar[i], 1);
+      mbar_init(&sfse_bar[i], 4);
+    }
     mbar_init(&accf_bar, 1);
     mbar_init(&acce_bar, C::EPI_WARPS);
     mbar_init(&drain_bar, 1);
@@ -564,46 +573,61 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   tc_fence_after();
   const uint32_t tmem = s_tmem_base;
 
-  // Producer pieces of one pipeline stage: the weight half (B tile and its
-  // scales) and the activation half (A tile and its scales), both completing
-  // on the stage's full barrier armed with the bytes of both.
-  auto stage_bytes = [&](const Unit& w, int kt) -> uint32_t {
-    const int steps = min(4, args.k_steps - 4 * kt);
+  // Two producers, two rings.  Operand tiles (warp 0): the weight half (B)
+  // and the activation half (A) of a stage complete on its full barrier.
+  // Scale atoms (warp 2): the weight scales (SFB) and activation scales
+  // (SFA) of a stage land in a ring of their own, which the scale writers
+  // release as soon as the atoms are in TMEM, so the scale factors of the
+  // next stages are in place before their operand tiles land.
+  uint8_t* sf_ring = smem + C::STAGES * C::STAGE_BYTES;
+  auto stage_steps = [&](int kt) { return min(4, args.k_steps - 4 * kt); };
+  auto sf_bytes = [&](const Unit& w, int kt) -> uint32_t {
     const int nrb = min(C::NRB, args.w_row_blocks - w.n * C::NRB);
-    return C::A_BYTES + C::B_BYTES + static_cast<uint32_t>(steps * 512 * (1 + nrb));
+    return static_cast<uint32_t>(stage_steps(kt) * 512 * (1 + nrb));
   };
   auto issue_weights = [&](int stage, const Unit& w, int kt) {
-    uint8_t* sb = smem + stage * C::STAGE_BYTES + C::A_BYTES;
-    uint8_t* ssfb = sb + C::B_BYTES + C::SFA_BYTES;
-    const int steps = min(4, args.k_steps - 4 * kt);
-    const int nrb = min(C::NRB, args.w_row_blocks - w.n * C::NRB);
-    tma_load_2d(sb, &tmB, &full_bar[stage], kt * 128, w.n * C::BN);
-    for (int rb = 0; rb < nrb; ++rb)
-      bulk_load(ssfb + rb * 2048, args.ws + (static_cast<size_t>(w.n * C::NRB + rb) * args.ka + 4 * kt) * 512,
-                steps * 512, &full_bar[stage]);
+    tma_load_2d(smem + stage * C::STAGE_BYTES + C::A_BYTES, &tmB, &full_bar[stage], kt * 128, w.n * C::BN);
   };
   auto issue_acts = [&](int stage, const Unit& w, int kt) {
-    uint8_t* sa = smem + stage * C::STAGE_BYTES;
-    uint8_t* ssfa = sa + C::A_BYTES + C::B_BYTES;
-    const int steps = min(4, args.k_steps - 4 * kt);
-    tma_load_2d(sa, &tmA, &full_bar[stage], kt * 128, w.m * kBM);
-    bulk_load(ssfa, args.xs + (static_cast<size_t>(w.m) * args.ka + 4 * kt) * 512, steps * 512, &full_bar[stage]);
+    tma_load_2d(smem + stage * C::STAGE_BYTES, &tmA, &full_bar[stage], kt * 128, w.m * kBM);
+  };
+  auto issue_weight_scales = [&](int slot, const Unit& w, int kt) {
+    uint8_t* ssfb = sf_ring + slot * C::SF_STAGE_BYTES + C::SFA_BYTES;
+    const int nrb = min(C::NRB, args.w_row_blocks - w.n * C::NRB);
+    for (int rb = 0; rb < nrb; ++rb)
+      bulk_load(ssfb + rb * 2048, args.ws + (static_cast<size_t>(w.n * C::NRB + rb) * args.ka + 4 * kt) * 512,
+                stage_steps(kt) * 512, &sfsf_bar[slot]);
+  };
+  auto issue_act_scales = [&](int slot, const Unit& w, int kt) {
+    bulk_load(sf_ring + slot * C::SF_STAGE_BYTES, args.xs + (static_cast<size_t>(w.m) * args.ka + 4 * kt) * 512,
+              stage_steps(kt) * 512, &sfsf_bar[slot]);
   };
 
   // Weights do not depend on the previous kernel on the stream (every
   // library kernel triggers its dependents only after its own dependency
   // wait, so all kernels two or more launches back, the weight quantizer
-  // among them, have completed): the first stages' weight halves stream in
-  // while the previous kernel (the activation quantizer) still runs.
-  int pre = 0;
-  uint32_t armed = 0;
+  // among them, have completed): the first stages' weight tiles and weight
+  // scales stream in while the previous kernel (the activation quantizer)
+  // still runs.
+  int pre = 0, sf_pre = 0;
+  uint32_t armed = 0, sf_armed = 0;
   if (warp == 0 && lane == 0) {
     for (int u = blockIdx.x; u < args.units && pre < C::STAGES; u += gridDim.x) {
       const Unit w = decode_unit(args, u);
       for (int kt = w.kt0; kt < w.kt1 && pre < C::STAGES; ++kt, ++pre) {
-        mbar_arrive_expect_tx(&full_bar[pre], stage_bytes(w, kt));
+        mbar_arrive_expect_tx(&full_bar[pre], C::A_BYTES + C::B_BYTES);
         armed |= 1u << pre;
         issue_weights(pre, w, kt);
+      }
+    }
+  }
+  if (warp == 2 && lane == 0) {
+    for (int u = blockIdx.x; u < args.units && sf_pre < C::SF_STAGES; u += gridDim.x) {
+      const Unit w = decode_unit(args, u);
+      for (int kt = w.kt0; kt < w.kt1 && sf_pre < C::SF_STAGES; ++kt, ++sf_pre) {
+        mbar_arrive_expect_tx(&sfsf_bar[sf_pre], sf_bytes(w, kt));
+        sf_armed |= 1u << sf_pre;
+        issue_weight_scales(sf_pre, w, kt);
       }
     }
   }
@@ -626,7 +650,7 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(&full_bar[stage], stage_bytes(w, kt));
+            mbar_arrive_expect_tx(&full_bar[stage], C::A_BYTES + C::B_BYTES);
             armed |= 1u << stage;
             armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
             issue_weights(stage, w, kt);
@@ -643,6 +667,43 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           if (armed & (1u << i)) {
             const long long t0 = clock64();
             while (!mbar_try_wait(&full_bar[i], (armed_phase >> i) & 1u) && clock64() - t0 < args.budget) {
+            }
+          }
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------ scale-atom producer
+    if (lane == 0) {
+      int slot = 0;
+      uint32_t phase = 0;
+      uint32_t armed_phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
+        const Unit w = decode_unit(args, u);
+        for (int kt = w.kt0; kt < w.kt1; ++kt, ++it) {
+          if (it >= sf_pre) {
+            if (!wait_or_abort(&sfse_bar[slot], phase ^ 1u, args.budget, &s_abort)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&sfsf_bar[slot], sf_bytes(w, kt));
+            sf_armed |= 1u << slot;
+            armed_phase = (armed_phase & ~(1u << slot)) | (phase << slot);
+            issue_weight_scales(slot, w, kt);
+          }
+          issue_act_scales(slot, w, kt);
+          if (++slot == C::SF_STAGES) {
+            slot = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        for (int i = 0; i < C::SF_STAGES; ++i)
+          if (sf_armed & (1u << i)) {
+            const long long t0 = clock64();
+            while (!mbar_try_wait(&sfsf_bar[i], (armed_phase >> i) & 1u) && clock64() - t0 < args.budget) {
             }
           }
       }
@@ -702,7 +763,7 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     regs_dec<48>();
     const int q = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-    int stage = 0;
+    int slot = 0;
     uint32_t phase = 0;
     int sfb = 0;
     uint32_t sf_phase = 0;
@@ -710,13 +771,13 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const Unit w = decode_unit(args, u);
       bool ok = true;
       for (int kt = w.kt0; kt < w.kt1; ++kt) {
-        if (!wait_or_abort(&full_bar[stage], phase, args.budget, &s_abort) ||
+        if (!wait_or_abort(&sfsf_bar[slot], phase, args.budget, &s_abort) ||
             !wait_or_abort(&sfe_bar[sfb], sf_phase ^ 1u, args.budget, &s_abort)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t ssfa = smem_u32(smem + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES);
+        const uint32_t ssfa = smem_u32(sf_ring + slot * C::SF_STAGE_BYTES);
         const uint32_t ssfb = ssfa + C::SFA_BYTES;
         const uint32_t dst = tmem + lane_base + C::SF_COL0 + sfb * C::SF_COLS;
         const int steps = min(4, args.k_steps - 4 * kt);
@@ -729,9 +790,12 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sff_bar[sfb]);
-        if (++stage == C::STAGES) {
-          stage = 0;
+        if (lane == 0) {
+          mbar_arrive(&sff_bar[sfb]);
+          mbar_arrive(&sfse_bar[slot]);  // the atoms are in TMEM: the slot may be refilled
+        }
+        if (++slot == C::SF_STAGES) {
+          slot = 0;
           phase ^= 1u;
         }
         if (++sfb == C::NSF) {
