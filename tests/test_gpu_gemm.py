@@ -140,12 +140,19 @@ def test_workspace_is_checked():
     assert ei.value.status == 7
 
 
-# Shapes with more than 74 output tiles of 128 x 256 take the wide-tile
-# prefill kernel (scale writers + early TMEM release); ragged M, N and K.
+# Shapes with more than 74 output tiles of 128 x 256 run without split-K.
+# With more than 128 rows they take the paired kernel (256 x 256 tiles over
+# the two CTAs of a cluster): ragged M (a tile whose odd CTA has no rows,
+# 777; rows 129-256, 200), ragged N (a tile whose odd CTA has no B rows,
+# 2568), ragged K, several tiles per CTA pair (9728, 19200).  With at most
+# 128 rows, the single-CTA kernel with its direct epilogue (100 rows).
 WIDE_CASES = [
     (1024, 2560, 1024, False),
     (1000, 2568, 336, True),
     (777, 4096, 512, True),
+    (1024, 9728, 512, False),
+    (200, 19200, 256, True),
+    (100, 19456, 256, True),
 ]
 
 

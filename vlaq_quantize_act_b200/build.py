@@ -26,7 +26,7 @@ FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std
 # per-warpgroup budgets they request add up to exactly this entry register
 # count times the block size, so ptxas must allocate exactly this many at
 # entry (fewer would make setmaxnreg.inc wait for registers that never free).
-ENTRY_REGISTERS = {"gemm_fp4_sfw_kernel": 128}
+ENTRY_REGISTERS = {"gemm_fp4_sfw_kernel": 128, "gemm_fp4_pair_kernel": 128}
 
 
 def _check_entry_registers(ptxas_log: str) -> None:

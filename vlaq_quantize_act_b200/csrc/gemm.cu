@@ -8,14 +8,17 @@
 // INT8 rounds each epilogue step once (fp32(acc), s_x s_w, product, residual
 // add), so its output is exact: one value, whatever the split or order.
 //
-// Two persistent, warp-specialised kernels, one CTA per SM, both fed by TMA
-// (2-D tiled loads of the packed codes with 128-byte swizzle) through a ring
-// of shared-memory stages, accumulating 128 x BN tiles in TMEM with
-// tcgen05.mma issued from one thread:
+// Persistent, warp-specialised kernels, one CTA per SM, fed by TMA (2-D
+// tiled loads of the packed codes with 128-byte swizzle) through a ring of
+// shared-memory stages, accumulating in TMEM with tcgen05.mma issued from
+// one thread:
 //   gemm_fp4_sfw_kernel  NVFP4, 128 x 256 tiles, kind::mxf4nvf4 with block-16
 //                        UE4M3 scale vectors that four warps write into TMEM;
 //                        split-K (decode shapes) reduced in-kernel by the
 //                        last split of each tile;
+//   gemm_fp4_pair_kernel NVFP4, 256 x 256 tiles over the two CTAs of a
+//                        cluster (paired MMA, cta_group::2): each SM streams
+//                        half of the weight tile; prefill shapes;
 //   gemm_fp8_kernel<BN, I8>  FP8 E4M3 (kind::f8f6f4, fp32 accumulators) or
 //                        INT8 (kind::i8, s32), 128 x 256 or 128 x 128 tiles
 //                        (double-buffered accumulator); split-K partials are
@@ -160,12 +163,13 @@ __device__ __forceinline__ float add_residual(float y, float r) {
   return I8 ? __fadd_rn(y, r) : y + r;
 }
 
-// Scale, residual add, bf16 round and store of one 32-column row segment.
+// Scaled, residual-added fp32 values of one 32-column row segment (row < M),
+// in place: r holds the accumulator bits on entry and the values' fp32 bits
+// on return (columns from N on are never stored).
 template <bool FP4, bool I8 = false>
-__device__ __forceinline__ void store_output(const GemmArgs& a, int row, int col0, float rs,
-                                             const uint32_t (&r)[32]) {
+__device__ __forceinline__ void epilogue_values(const GemmArgs& a, int row, int col0, float rs, uint32_t (&r)[32]) {
   const bool full = col0 + 32 <= a.N;
-  float y[32];
+  float* y = reinterpret_cast<float*>(r);
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
     if constexpr (FP4) {
@@ -195,6 +199,16 @@ __device__ __forceinline__ void store_output(const GemmArgs& a, int row, int col
         if (col0 + j < a.N) y[j] = add_residual<I8>(y[j], __bfloat162float(a.residual[base + j]));
     }
   }
+}
+
+// Scale, residual add, bf16 round and store of one 32-column row segment
+// (r is overwritten).
+template <bool FP4, bool I8 = false>
+__device__ __forceinline__ void store_output(const GemmArgs& a, int row, int col0, float rs, uint32_t (&r)[32]) {
+  const bool full = col0 + 32 <= a.N;
+  epilogue_values<FP4, I8>(a, row, col0, rs, r);
+  const float* y = reinterpret_cast<const float*>(r);
+  const size_t base = static_cast<size_t>(row) * a.N + col0;
   if (full) {
     // two 32-byte stores: each thread writes whole sectors of its row
     uint32_t pk[16];
@@ -875,6 +889,430 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   }
 }
 
+// NVFP4 GEMM over CTA pairs: 256 x 256 tiles computed by the paired MMA
+// (tcgen05.mma.cta_group::2) across the two CTAs of a cluster.  CTA r of the
+// pair loads rows [128 r, 128 r + 128) of the A tile and of the B tile, so
+// each SM streams half of the weight tile: 256 operand rows per 128 x 256
+// outputs instead of 384 on one SM.  Each CTA writes the scale factors of
+// its own 128 A rows and of all 256 B rows into its own TMEM (the layout
+// of the single-CTA kernel), reads its own 128 accumulator rows and stores
+// them through shared memory with TMA tile stores.  The leader (even CTA)
+// issues the MMAs.  The issuing thread waits once and commits once per stage
+// (an MMA issue returns only about when the tensor core takes it, so every
+// barrier operation of that thread is idle tensor-core time): the leader's
+// full barrier of a stage completes on the operand bytes of both CTAs and
+// the arrivals of both CTAs' scale writers, and one commit to the stage's
+// empty barrier in both CTAs frees the operand stage and the stage's TMEM
+// scale buffer.  Direct epilogue only (used when the output tiles already
+// fill the GPU).
+struct PairCfg {
+  static constexpr int BM = 256;                 // tile rows over the pair
+  static constexpr int BN = 256;
+  static constexpr int A_BYTES = 128 * 128;      // this CTA's 128 A rows of one stage
+  static constexpr int B_BYTES = 128 * 128;      // this CTA's 128 B rows
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = 5;
+  static constexpr int SFA_BYTES = 4 * 512;
+  static constexpr int SFB_BYTES = 2 * 4 * 512;  // both 128-row blocks of the B tile
+  static constexpr int SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;
+  static constexpr int SF_STAGES = 4;
+  static constexpr int NSF = 4;                  // TMEM scale buffers (fewer than STAGES)
+  static constexpr int SF_COLS = 16 + 32;        // per buffer: 16 (A) + 32 (B)
+  static constexpr int SF_COL0 = BN;             // after the accumulator
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int OUT_BOX_COLS = 64;        // output store box: 32 rows x 64 bf16 (128-byte rows)
+  static constexpr int OUT_BYTES = 32 * OUT_BOX_COLS * 2;  // one box per epilogue warp
+  static constexpr int OUT_OFFSET = STAGES * STAGE_BYTES + SF_STAGES * SF_STAGE_BYTES;
+  static constexpr int SMEM_BYTES = OUT_OFFSET + EPI_WARPS * OUT_BYTES + 1024;
+  static constexpr int THREADS = 512;
+  static constexpr uint32_t IDESC =
+      (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+  static_assert(OUT_OFFSET % 1024 == 0 && OUT_BYTES % 1024 == 0, "128-byte swizzle atoms of the output boxes");
+  static_assert(SF_COL0 + NSF * SF_COLS <= kTmemCols, "TMEM budget");
+  // a scale buffer is rewritten for stage i once stage i - NSF is consumed;
+  // with NSF < STAGES that empty phase cannot be overtaken before it is
+  // waited on, and the writers' arrival for stage i lands in stage i's phase
+  static_assert(NSF < STAGES, "scale buffers recycle on the operand stages' empty barriers");
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+// Bounded wait for the pair kernel: gives up when either CTA of the pair
+// aborted, and on running out raises the abort flag of both.
+__device__ __forceinline__ bool pair_wait(uint64_t* bar, uint32_t parity, long long budget, volatile int* abort_flag,
+                                          uint32_t peer_abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > budget) {
+      raise_abort(abort_flag);
+      st_shared_cluster_u32(peer_abort, 1u);
+      return false;
+    }
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
+gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmY, const GemmArgs args) {
+  using C = PairCfg;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[C::STAGES];     // leader: operands and scale factors of both CTAs
+  __shared__ __align__(8) uint64_t empty_bar[C::STAGES];    // stage consumed (leader's commit)
+  __shared__ __align__(8) uint64_t sfsf_bar[C::SF_STAGES];  // scale atoms landed
+  __shared__ __align__(8) uint64_t sfse_bar[C::SF_STAGES];  // scale atoms copied to TMEM
+  __shared__ __align__(8) uint64_t accf_bar;                // accumulator complete (leader's commit)
+  __shared__ __align__(8) uint64_t acce_bar;                // leader: both CTAs' accumulators read
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t s_tmem_base;
+  __shared__ volatile int s_abort;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int wg = warp >> 2;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int pairs = static_cast<int>(gridDim.x >> 1);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&full_bar[i], 1 + 8);  // the leader's producer + four scale writers per CTA
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < C::SF_STAGES; ++i) {
+      mbar_init(&sfsf_bar[i], 1);
+      mbar_init(&sfse_bar[i], 4);
+    }
+    mbar_init(&accf_bar, 1);
+    mbar_init(&acce_bar, 2 * C::EPI_WARPS);
+    mbar_init(&drain_bar, 1);
+    s_abort = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmY);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&s_tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();  // both CTAs' barriers are initialised before either CTA signals the other's
+  tc_fence_after();
+  const uint32_t tmem = s_tmem_base;
+  const uint32_t peer_abort = mapa_shared(smem_u32(const_cast<int*>(&s_abort)), rank ^ 1u);
+  auto leader_bar = [&](uint64_t* bar) { return mapa_shared(smem_u32(bar), 0u); };
+
+  uint8_t* sf_ring = smem + C::STAGES * C::STAGE_BYTES;
+  const int x_row_blocks = (args.M + 127) / 128;
+  auto stage_steps = [&](int kt) { return min(4, args.k_steps - 4 * kt); };
+  auto own_a_block = [&](const Unit& w) { return 2 * w.m + static_cast<int>(rank); };
+  auto sf_bytes = [&](const Unit& w, int kt) -> uint32_t {
+    const int nrb = min(2, args.w_row_blocks - 2 * w.n);
+    const int has_a = own_a_block(w) < x_row_blocks ? 1 : 0;
+    return static_cast<uint32_t>(stage_steps(kt) * 512 * (has_a + nrb));
+  };
+  auto issue_weights = [&](int stage, const Unit& w, int kt) {
+    tma_load_2d_pair(smem + stage * C::STAGE_BYTES + C::A_BYTES, &tmB, leader_bar(&full_bar[stage]), kt * 128,
+                     w.n * C::BN + 128 * static_cast<int>(rank));
+  };
+  auto issue_acts = [&](int stage, const Unit& w, int kt) {
+    tma_load_2d_pair(smem + stage * C::STAGE_BYTES, &tmA, leader_bar(&full_bar[stage]), kt * 128,
+                     w.m * C::BM + 128 * static_cast<int>(rank));
+  };
+  auto issue_weight_scales = [&](int slot, const Unit& w, int kt) {
+    uint8_t* ssfb = sf_ring + slot * C::SF_STAGE_BYTES + C::SFA_BYTES;
+    const int nrb = min(2, args.w_row_blocks - 2 * w.n);
+    for (int rb = 0; rb < nrb; ++rb)
+      bulk_load(ssfb + rb * 2048, args.ws + (static_cast<size_t>(2 * w.n + rb) * args.ka + 4 * kt) * 512,
+                stage_steps(kt) * 512, &sfsf_bar[slot]);
+  };
+  auto issue_act_scales = [&](int slot, const Unit& w, int kt) {
+    const int ab = own_a_block(w);
+    if (ab < x_row_blocks)
+      bulk_load(sf_ring + slot * C::SF_STAGE_BYTES, args.xs + (static_cast<size_t>(ab) * args.ka + 4 * kt) * 512,
+                stage_steps(kt) * 512, &sfsf_bar[slot]);
+  };
+
+  // Weights (and their scale atoms) do not depend on the previous kernel on
+  // the stream: the first stages stream in before the dependency wait.
+  int pre = 0, sf_pre = 0;
+  uint32_t armed = 0, sf_armed = 0;
+  if (warp == 0 && lane == 0) {
+    for (int u = pair; u < args.units && pre < C::STAGES; u += pairs) {
+      const Unit w = decode_unit(args, u);
+      for (int kt = w.kt0; kt < w.kt1 && pre < C::STAGES; ++kt, ++pre) {
+        if (rank == 0) mbar_arrive_expect_tx(&full_bar[pre], 2 * C::STAGE_BYTES);
+        armed |= 1u << pre;
+        issue_weights(pre, w, kt);
+      }
+    }
+  }
+  if (warp == 2 && lane == 0) {
+    for (int u = pair; u < args.units && sf_pre < C::SF_STAGES; u += pairs) {
+      const Unit w = decode_unit(args, u);
+      for (int kt = w.kt0; kt < w.kt1 && sf_pre < C::SF_STAGES; ++kt, ++sf_pre) {
+        mbar_arrive_expect_tx(&sfsf_bar[sf_pre], sf_bytes(w, kt));
+        sf_armed |= 1u << sf_pre;
+        issue_weight_scales(sf_pre, w, kt);
+      }
+    }
+  }
+  griddep_wait();
+  griddep_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------- operand producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed_phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int u = pair; u < args.units && ok; u += pairs) {
+        const Unit w = decode_unit(args, u);
+        for (int kt = w.kt0; kt < w.kt1; ++kt, ++it) {
+          if (it >= pre) {
+            if (!pair_wait(&empty_bar[stage], phase ^ 1u, args.budget, &s_abort, peer_abort)) {
+              ok = false;
+              break;
+            }
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * C::STAGE_BYTES);
+            armed |= 1u << stage;
+            armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+            issue_weights(stage, w, kt);
+          }
+          issue_acts(stage, w, kt);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (ok) {
+        // every stage released: the leader's last commits to this CTA have landed
+        for (int i = 0; i < C::STAGES && ok; ++i) {
+          ok = pair_wait(&empty_bar[stage], phase ^ 1u, args.budget, &s_abort, peer_abort);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      } else if (rank == 0) {
+        for (int i = 0; i < C::STAGES; ++i)
+          if (armed & (1u << i)) {
+            const long long t0 = clock64();
+            while (!mbar_try_wait(&full_bar[i], (armed_phase >> i) & 1u) && clock64() - t0 < args.budget) {
+            }
+          }
+      } else {
+        // the peer cannot observe the leader's barriers: give its copies in
+        // flight time to land before the pair's final barrier
+        const long long t0 = clock64();
+        while (clock64() - t0 < (1ll << 21)) {
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------- scale-atom producer (both CTAs)
+    if (lane == 0) {
+      int slot = 0;
+      uint32_t phase = 0;
+      uint32_t armed_phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int u = pair; u < args.units && ok; u += pairs) {
+        const Unit w = decode_unit(args, u);
+        for (int kt = w.kt0; kt < w.kt1; ++kt, ++it) {
+          if (it >= sf_pre) {
+            if (!pair_wait(&sfse_bar[slot], phase ^ 1u, args.budget, &s_abort, peer_abort)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&sfsf_bar[slot], sf_bytes(w, kt));
+            sf_armed |= 1u << slot;
+            armed_phase = (armed_phase & ~(1u << slot)) | (phase << slot);
+            issue_weight_scales(slot, w, kt);
+          }
+          issue_act_scales(slot, w, kt);
+          if (++slot == C::SF_STAGES) {
+            slot = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        for (int i = 0; i < C::SF_STAGES; ++i)
+          if (sf_armed & (1u << i)) {
+            const long long t0 = clock64();
+            while (!mbar_try_wait(&sfsf_bar[i], (armed_phase >> i) & 1u) && clock64() - t0 < args.budget) {
+            }
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (leader)
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int sfb = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int u = pair; u < args.units && ok; u += pairs) {
+        const Unit w = decode_unit(args, u);
+        if (!pair_wait(&acce_bar, acc_phase ^ 1u, args.budget, &s_abort, peer_abort)) break;
+        tc_fence_after();
+        for (int kt = w.kt0; kt < w.kt1; ++kt) {
+          if (!pair_wait(&full_bar[stage], phase, args.budget, &s_abort, peer_abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sa + C::A_BYTES);
+          const uint32_t sf = tmem + C::SF_COL0 + sfb * C::SF_COLS;
+          const int steps = stage_steps(kt);
+          for (int j = 0; j < steps; ++j)
+            mma_mxf4nvf4_pair(tmem, sdesc_kmajor_sw128(a0 + 32 * j), sdesc_kmajor_sw128(b0 + 32 * j), C::IDESC,
+                              sf + 4 * j, sf + 16 + 8 * j, (kt > w.kt0 || j > 0) ? 1u : 0u);
+          umma_commit_pair(&empty_bar[stage], 0x3);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          if (++sfb == C::NSF) sfb = 0;
+        }
+        if (!ok) break;
+        umma_commit_pair(&accf_bar, 0x3);
+        acc_phase ^= 1u;
+      }
+      umma_commit_pair(&drain_bar, 0x1);
+      const long long t0 = clock64();
+      while (!mbar_try_wait(&drain_bar, 0) && clock64() - t0 < 4 * args.budget + 1000000) {
+      }
+    }
+  } else if (wg == 3) {
+    // ----------------------------------------- scale writers (both CTAs)
+    // Stage i (counted over this pair's tiles) goes to TMEM scale buffer
+    // i % NSF once stage i - NSF is consumed; the writers then arrive on the
+    // leader's full barrier of stage i.
+    regs_dec<48>();
+    const int q = warp & 3;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+    int slot = 0;
+    uint32_t phase = 0;
+    int i = 0;
+    bool ok = true;
+    for (int u = pair; u < args.units && ok; u += pairs) {
+      const Unit w = decode_unit(args, u);
+      for (int kt = w.kt0; kt < w.kt1; ++kt, ++i) {
+        const int prev = i - C::NSF;
+        if (!pair_wait(&sfsf_bar[slot], phase, args.budget, &s_abort, peer_abort) ||
+            (prev >= 0 && !pair_wait(&empty_bar[prev % C::STAGES], static_cast<uint32_t>(prev / C::STAGES) & 1u,
+                                     args.budget, &s_abort, peer_abort))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ssfa = smem_u32(sf_ring + slot * C::SF_STAGE_BYTES);
+        const uint32_t ssfb = ssfa + C::SFA_BYTES;
+        const uint32_t dst = tmem + lane_base + C::SF_COL0 + (i % C::NSF) * C::SF_COLS;
+        const int steps = stage_steps(kt);
+        for (int j = 0; j < steps; ++j) {
+          tmem_st_32x32b_x4(dst + 4 * j, ld_shared_v4(ssfa + 512 * j + 16 * lane));
+#pragma unroll
+          for (int rb = 0; rb < 2; ++rb)
+            tmem_st_32x32b_x4(dst + 16 + 8 * j + 4 * rb, ld_shared_v4(ssfb + rb * 2048 + 512 * j + 16 * lane));
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_cluster(leader_bar(&full_bar[i % C::STAGES]));
+          mbar_arrive(&sfse_bar[slot]);
+        }
+        if (++slot == C::SF_STAGES) {
+          slot = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    tmem_st_wait();
+  } else if (wg == 1 || wg == 2) {
+    // ------------------------------------------------- epilogue (both CTAs)
+    // Warp (q, h) owns TMEM lanes 32q..32q+31 (tile rows) and columns
+    // 128h..128h+127; each 64-column box is scaled, rounded to bf16, written
+    // to the warp's staging box in the 128-byte swizzle layout and stored
+    // with one TMA tile store (rows from M and columns from N are clipped).
+    regs_inc<168>();
+    const int e = warp - 4;
+    const int q = warp & 3;
+    const int h = e >> 2;
+    const uint32_t box = smem_u32(smem + C::OUT_OFFSET + e * C::OUT_BYTES);
+    uint32_t acc_phase = 0;
+    for (int u = pair; u < args.units; u += pairs) {
+      const Unit w = decode_unit(args, u);
+      if (!pair_wait(&accf_bar, acc_phase, args.budget, &s_abort, peer_abort)) break;
+      tc_fence_after();
+      const int row0 = w.m * C::BM + 128 * static_cast<int>(rank) + 32 * q;
+      const int row = row0 + lane;
+      const bool row_ok = row < args.M;
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(128 * h);
+      __syncwarp();
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tbase + 32 * c, r[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_bar(&acce_bar));
+      acc_phase ^= 1u;
+      const float rs = row_ok ? args.xg[row] * args.wg[0] : 0.0f;
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        const int col0 = w.n * C::BN + 128 * h + C::OUT_BOX_COLS * b;
+        if (col0 >= args.N || row0 >= args.M) continue;  // box wholly outside the output (warp-uniform)
+        if (lane == 0) bulk_wait_group_read0();          // the previous store has read the staging box
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if (row_ok) epilogue_values<true>(args, row, col0 + 32 * c, rs, r[2 * b + c]);
+          const float* y = reinterpret_cast<const float*>(r[2 * b + c]);  // rows from M on: clipped by the store
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {  // 16-byte chunk 4c + j of this row, swizzled by row % 8
+            const uint32_t chunk = static_cast<uint32_t>((4 * c + j) ^ (lane & 7));
+            st_shared_v4(box + 128 * lane + 16 * chunk, pack_bf16x2(y[8 * j], y[8 * j + 1]),
+                         pack_bf16x2(y[8 * j + 2], y[8 * j + 3]), pack_bf16x2(y[8 * j + 4], y[8 * j + 5]),
+                         pack_bf16x2(y[8 * j + 6], y[8 * j + 7]));
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmY, smem + C::OUT_OFFSET + e * C::OUT_BYTES, col0, row0);
+          bulk_commit_group();
+        }
+      }
+    }
+    if (lane == 0) bulk_wait_group0();
+  }
+
+  // Neither CTA leaves (or frees its TMEM) while the other may still signal
+  // it or the paired MMAs may still touch its shared memory or TMEM.
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
 // Split-K reduction + epilogue: fixed split order, same scaling as the
 // direct epilogue (INT8: exact s32 sums, then the INT8 epilogue steps).
 // 8 outputs per thread.
@@ -962,6 +1400,21 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t r
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 output [rows, cols] for TMA tile stores: box 64 columns x 32 rows
+// (128-byte rows), 128-byte swizzle.  Needs a 16-byte aligned base and
+// cols % 8 == 0.
+bool make_out_map(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Launch arguments shared by both GEMM kernels (BN: tile width).
 GemmArgs make_args(bool fp4, int BN, const uint8_t* xs, const float* xg, const uint8_t* ws, const float* wg,
                    const void* residual, void* Y, int64_t M, int64_t N, int64_t K, void* workspace,
@@ -1008,6 +1461,54 @@ cudaError_t run_fp4(const uint8_t* xq, const uint8_t* xs, const float* xg, const
       cudaFuncSetAttribute(gemm_fp4_sfw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SfwCfg::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   return launch_pdl(gemm_fp4_sfw_kernel, dim3(grid), dim3(SfwCfg::THREADS), SfwCfg::SMEM_BYTES, s, ta, tb, a);
+}
+
+// Clusters of gemm_fp4_pair_kernel that fit on the device at once (cached
+// per device; half the SMs when the query fails).
+int pair_clusters_resident() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return device_sm_count() / 2;
+  static int cache[64] = {0};
+  if (dev < 64 && cache[dev]) return cache[dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned int>(device_sm_count()));
+  cfg.blockDim = dim3(PairCfg::THREADS);
+  cfg.dynamicSmemBytes = PairCfg::SMEM_BYTES;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_fp4_pair_kernel, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = device_sm_count() / 2;
+  }
+  if (dev < 64) cache[dev] = n;
+  return n;
+}
+
+// NVFP4 over CTA pairs: 256 x 256 tiles, direct epilogue through TMA
+// stores.  An output the store map cannot describe (base not 16-byte
+// aligned) runs the single-CTA kernel instead.
+cudaError_t run_fp4_pair(const uint8_t* xq, const uint8_t* xs, const float* xg, const uint8_t* wq, const uint8_t* ws,
+                         const float* wg, const void* residual, void* Y, int64_t M, int64_t N, int64_t K,
+                         void* workspace, const GemmPlan& plan, long long budget, cudaStream_t s) {
+  const int64_t pitch = nvfp4_code_pitch(K);
+  CUtensorMap ta, tb, ty;
+  if (!make_out_map(&ty, Y, static_cast<uint64_t>(N), static_cast<uint64_t>(M)))
+    return run_fp4(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
+  if (!make_map(&ta, xq, static_cast<uint64_t>(pitch), static_cast<uint64_t>(M), static_cast<uint64_t>(pitch), 128) ||
+      !make_map(&tb, wq, static_cast<uint64_t>(pitch), static_cast<uint64_t>(N), static_cast<uint64_t>(pitch), 128))
+    return cudaErrorInvalidValue;
+  GemmArgs a = make_args(true, PairCfg::BN, xs, xg, ws, wg, residual, Y, M, N, K, nullptr, plan, budget);
+  a.m_tiles = static_cast<int>((M + PairCfg::BM - 1) / PairCfg::BM);
+  a.splits = 1;
+  a.units = a.m_tiles * a.n_tiles;
+  cudaError_t e =
+      cudaFuncSetAttribute(gemm_fp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  int pairs = pair_clusters_resident();
+  if (plan.grid / 2 < pairs) pairs = plan.grid / 2;
+  if (a.units < pairs) pairs = a.units;
+  if (pairs < 1) pairs = 1;
+  return launch_pdl(gemm_fp4_pair_kernel, dim3(static_cast<unsigned int>(2 * pairs)), dim3(PairCfg::THREADS),
+                    PairCfg::SMEM_BYTES, s, ta, tb, ty, a);
 }
 
 // FP8 / INT8: gemm_fp8_kernel<BN, I8>, then the ordered split-K reduction
@@ -1068,6 +1569,14 @@ GemmPlan plan_gemm(bool fp4, int64_t M, int64_t N, int64_t K, int num_sms) {
     const int64_t units = tiles * splits;
     p.grid = static_cast<int>(units < num_sms ? units : num_sms);
     p.ws_bytes = splits > 1 ? kSplitCounterBytes + splitk_partial_bytes(splits, M, N) : 0;
+    // Tiles that fill the GPU and more than 128 rows: 256 x 256 tiles over
+    // CTA pairs, each SM streaming half of the weight tile.
+    if (splits == 1 && M > kBM) {
+      const int64_t pair_units = ((M + 255) / 256) * ((N + 255) / 256);
+      const int64_t pairs = num_sms / 2;
+      p.pair = true;
+      p.grid = static_cast<int>(2 * (pair_units < pairs ? pair_units : pairs));
+    }
     return p;
   }
   // Wide tiles halve the scale-factor copies per FLOP and the A re-reads;
@@ -1102,6 +1611,8 @@ cudaError_t launch_linear(bool fp4, const uint8_t* xq, const uint8_t* xs, const 
                           cudaStream_t s) {
   (void)ws_bytes;
   if (fp4 && plan.bn == 0) return launch_gemv_nvfp4(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, s);
+  if (fp4 && plan.pair)
+    return run_fp4_pair(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
   if (fp4) return run_fp4(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
   if (plan.bn == 256) return run_fp8<256, false>(xq, xg, wq, wg, residual, Y, M, N, K, workspace, plan, budget, s);
   return run_fp8<128, false>(xq, xg, wq, wg, residual, Y, M, N, K, workspace, plan, budget, s);

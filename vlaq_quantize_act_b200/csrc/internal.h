@@ -48,10 +48,11 @@ cudaError_t launch_scales_to_rowmajor(const uint8_t* in, uint8_t* out, int64_t r
 
 // ---- GEMM (gemm.cu)
 struct GemmPlan {
-  int bn;          // tile width along N (0: the few-row CUDA-core kernel)
-  int splits;      // split-K factor (1 = direct epilogue)
-  int grid;        // persistent CTAs
-  size_t ws_bytes; // fp32 partials needed when splits > 1
+  int bn;            // tile width along N (0: the few-row CUDA-core kernel)
+  int splits;        // split-K factor (1 = direct epilogue)
+  int grid;          // persistent CTAs
+  size_t ws_bytes;   // fp32 partials needed when splits > 1
+  bool pair = false; // NVFP4: 256 x 256 tiles over CTA pairs (paired MMA)
 };
 GemmPlan plan_gemm(bool fp4, int64_t M, int64_t N, int64_t K, int num_sms);
 // Split-K workspace layout: the NVFP4 per-tile arrival counters occupy the
