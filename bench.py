@@ -674,7 +674,7 @@ def prefill_section(vq, data, args, dist_on, device, peaks, world):
                    "l2": "inputs larger than L2 (per-step working set ~294 MB)", "graph": True},
         "roofline": {"bound": "tensor", "achieved": g_ach, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": g_ach / fp4_peak, "traffic": traffic,
-                     "kernel": "gemm_fp4_sfw_kernel gate_up 1024x37888x3584 (2MNK = 278.1 GFLOP per launch)",
+                     "kernel": "gemm_fp4_pair_kernel gate_up 1024x37888x3584 (2MNK = 278.1 GFLOP per launch)",
                      "all_gemms_tflops": gemm_all, "all_gemms_frac": gemm_all / fp4_peak,
                      "timing": f"CUDA events in a {tmode} capture of the step",
                      "peak_note": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 4 (nominal FP4:BF16)"},
