@@ -144,14 +144,19 @@ def test_workspace_is_checked():
 # With more than 128 rows they take the paired kernel (256 x 256 tiles over
 # the two CTAs of a cluster): ragged M (a tile whose odd CTA has no rows,
 # 777; rows 129-256, 200), ragged N (a tile whose odd CTA has no B rows,
-# 2568), ragged K, several tiles per CTA pair (9728, 19200).  With at most
-# 128 rows, the single-CTA kernel with its direct epilogue (100 rows).
+# 2568), several tiles per CTA pair (9728, 19200).  K % 256 == 0 runs two
+# K-chunks per stage (an odd chunk count, 1024 + 256 ... 256, leaves the
+# last stage half outside K); other K one chunk per stage with TMA stores
+# (336, 320).  With at most 128 rows, the single-CTA kernel with its direct
+# epilogue (100 rows).
 WIDE_CASES = [
     (1024, 2560, 1024, False),
     (1000, 2568, 336, True),
     (777, 4096, 512, True),
     (1024, 9728, 512, False),
     (200, 19200, 256, True),
+    (512, 19200, 320, False),
+    (384, 9728, 1280, True),
     (100, 19456, 256, True),
 ]
 

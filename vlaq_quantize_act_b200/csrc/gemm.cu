@@ -905,25 +905,37 @@ gemm_fp4_sfw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 // empty barrier in both CTAs frees the operand stage and the stage's TMEM
 // scale buffer.  Direct epilogue only (used when the output tiles already
 // fill the GPU).
+// CH: 128-byte K-chunks per stage.  CH = 2 (K = 512 per stage) loads each
+// row's two chunks with one 3-D TMA box; the TMA engine moves about twice
+// the bytes per load instruction, and the MMA thread's one wait and one
+// commit cover eight MMAs.  It needs rows of whole chunks (K % 256 == 0);
+// other K run CH = 1 with 2-D boxes.  CH = 1 stages the output for TMA
+// stores; CH = 2 has no shared memory left for that and stores rows directly.
+template <int CH>
 struct PairCfg {
   static constexpr int BM = 256;                 // tile rows over the pair
   static constexpr int BN = 256;
-  static constexpr int A_BYTES = 128 * 128;      // this CTA's 128 A rows of one stage
-  static constexpr int B_BYTES = 128 * 128;      // this CTA's 128 B rows
+  static constexpr int CHUNK_BYTES = 128 * 128;  // one K-chunk of this CTA's 128 rows
+  static constexpr int A_BYTES = CH * CHUNK_BYTES;
+  static constexpr int B_BYTES = CH * CHUNK_BYTES;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = 5;
-  static constexpr int SFA_BYTES = 4 * 512;
-  static constexpr int SFB_BYTES = 2 * 4 * 512;  // both 128-row blocks of the B tile
+  static constexpr int STEPS = 4 * CH;           // MMAs (K = 64) per stage
+  static constexpr int STAGES = CH == 1 ? 5 : 3;
+  static constexpr int SFA_BYTES = STEPS * 512;
+  static constexpr int SFB_ROW_BYTES = STEPS * 512;  // one 128-row block of the B tile
+  static constexpr int SFB_BYTES = 2 * SFB_ROW_BYTES;
   static constexpr int SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;
-  static constexpr int SF_STAGES = 4;
-  static constexpr int NSF = 4;                  // TMEM scale buffers (fewer than STAGES)
-  static constexpr int SF_COLS = 16 + 32;        // per buffer: 16 (A) + 32 (B)
+  static constexpr int SF_STAGES = CH == 1 ? 4 : 2;
+  static constexpr int NSF = CH == 1 ? 4 : 2;   // TMEM scale buffers (fewer than STAGES)
+  static constexpr int SFB_COL = 4 * STEPS;      // B scale columns after the A ones
+  static constexpr int SF_COLS = 12 * STEPS;     // per buffer: 4 (A) + 8 (B) per MMA
   static constexpr int SF_COL0 = BN;             // after the accumulator
   static constexpr int EPI_WARPS = 8;
+  static constexpr bool TMA_STORE = CH == 1;
   static constexpr int OUT_BOX_COLS = 64;        // output store box: 32 rows x 64 bf16 (128-byte rows)
   static constexpr int OUT_BYTES = 32 * OUT_BOX_COLS * 2;  // one box per epilogue warp
   static constexpr int OUT_OFFSET = STAGES * STAGE_BYTES + SF_STAGES * SF_STAGE_BYTES;
-  static constexpr int SMEM_BYTES = OUT_OFFSET + EPI_WARPS * OUT_BYTES + 1024;
+  static constexpr int SMEM_BYTES = OUT_OFFSET + (TMA_STORE ? EPI_WARPS * OUT_BYTES : 0) + 1024;
   static constexpr int THREADS = 512;
   static constexpr uint32_t IDESC =
       (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
@@ -954,10 +966,11 @@ __device__ __forceinline__ bool pair_wait(uint64_t* bar, uint32_t parity, long l
   }
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
+template <int CH>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<CH>::THREADS, 1)
 gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmY, const GemmArgs args) {
-  using C = PairCfg;
+  using C = PairCfg<CH>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[C::STAGES];     // leader: operands and scale factors of both CTAs
   __shared__ __align__(8) uint64_t empty_bar[C::STAGES];    // stage consumed (leader's commit)
@@ -1010,33 +1023,40 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
 
   uint8_t* sf_ring = smem + C::STAGES * C::STAGE_BYTES;
   const int x_row_blocks = (args.M + 127) / 128;
-  auto stage_steps = [&](int kt) { return min(4, args.k_steps - 4 * kt); };
+  auto stage_steps = [&](int kt) { return min(C::STEPS, args.k_steps - C::STEPS * kt); };
   auto own_a_block = [&](const Unit& w) { return 2 * w.m + static_cast<int>(rank); };
   auto sf_bytes = [&](const Unit& w, int kt) -> uint32_t {
     const int nrb = min(2, args.w_row_blocks - 2 * w.n);
     const int has_a = own_a_block(w) < x_row_blocks ? 1 : 0;
     return static_cast<uint32_t>(stage_steps(kt) * 512 * (has_a + nrb));
   };
+  auto load = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int kt, int row) {
+    if constexpr (CH == 1)
+      tma_load_2d_pair(dst, map, leader_bar(bar), kt * 128, row);
+    else
+      tma_load_3d_pair(dst, map, leader_bar(bar), 0, row, kt * CH);
+  };
   auto issue_weights = [&](int stage, const Unit& w, int kt) {
-    tma_load_2d_pair(smem + stage * C::STAGE_BYTES + C::A_BYTES, &tmB, leader_bar(&full_bar[stage]), kt * 128,
-                     w.n * C::BN + 128 * static_cast<int>(rank));
+    load(smem + stage * C::STAGE_BYTES + C::A_BYTES, &tmB, &full_bar[stage], kt,
+         w.n * C::BN + 128 * static_cast<int>(rank));
   };
   auto issue_acts = [&](int stage, const Unit& w, int kt) {
-    tma_load_2d_pair(smem + stage * C::STAGE_BYTES, &tmA, leader_bar(&full_bar[stage]), kt * 128,
-                     w.m * C::BM + 128 * static_cast<int>(rank));
+    load(smem + stage * C::STAGE_BYTES, &tmA, &full_bar[stage], kt, w.m * C::BM + 128 * static_cast<int>(rank));
   };
   auto issue_weight_scales = [&](int slot, const Unit& w, int kt) {
     uint8_t* ssfb = sf_ring + slot * C::SF_STAGE_BYTES + C::SFA_BYTES;
     const int nrb = min(2, args.w_row_blocks - 2 * w.n);
     for (int rb = 0; rb < nrb; ++rb)
-      bulk_load(ssfb + rb * 2048, args.ws + (static_cast<size_t>(2 * w.n + rb) * args.ka + 4 * kt) * 512,
-                stage_steps(kt) * 512, &sfsf_bar[slot]);
+      bulk_load(ssfb + rb * C::SFB_ROW_BYTES,
+                args.ws + (static_cast<size_t>(2 * w.n + rb) * args.ka + C::STEPS * kt) * 512, stage_steps(kt) * 512,
+                &sfsf_bar[slot]);
   };
   auto issue_act_scales = [&](int slot, const Unit& w, int kt) {
     const int ab = own_a_block(w);
     if (ab < x_row_blocks)
-      bulk_load(sf_ring + slot * C::SF_STAGE_BYTES, args.xs + (static_cast<size_t>(ab) * args.ka + 4 * kt) * 512,
-                stage_steps(kt) * 512, &sfsf_bar[slot]);
+      bulk_load(sf_ring + slot * C::SF_STAGE_BYTES,
+                args.xs + (static_cast<size_t>(ab) * args.ka + C::STEPS * kt) * 512, stage_steps(kt) * 512,
+                &sfsf_bar[slot]);
   };
 
   // Weights (and their scale atoms) do not depend on the previous kernel on
@@ -1177,9 +1197,11 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
           const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sa + C::A_BYTES);
           const uint32_t sf = tmem + C::SF_COL0 + sfb * C::SF_COLS;
           const int steps = stage_steps(kt);
-          for (int j = 0; j < steps; ++j)
-            mma_mxf4nvf4_pair(tmem, sdesc_kmajor_sw128(a0 + 32 * j), sdesc_kmajor_sw128(b0 + 32 * j), C::IDESC,
-                              sf + 4 * j, sf + 16 + 8 * j, (kt > w.kt0 || j > 0) ? 1u : 0u);
+          for (int j = 0; j < steps; ++j) {
+            const uint32_t off = (j >> 2) * C::CHUNK_BYTES + 32 * (j & 3);  // chunk, then 64 K within it
+            mma_mxf4nvf4_pair(tmem, sdesc_kmajor_sw128(a0 + off), sdesc_kmajor_sw128(b0 + off), C::IDESC, sf + 4 * j,
+                              sf + C::SFB_COL + 8 * j, (kt > w.kt0 || j > 0) ? 1u : 0u);
+          }
           umma_commit_pair(&empty_bar[stage], 0x3);
           if (++stage == C::STAGES) {
             stage = 0;
@@ -1227,7 +1249,8 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
           tmem_st_32x32b_x4(dst + 4 * j, ld_shared_v4(ssfa + 512 * j + 16 * lane));
 #pragma unroll
           for (int rb = 0; rb < 2; ++rb)
-            tmem_st_32x32b_x4(dst + 16 + 8 * j + 4 * rb, ld_shared_v4(ssfb + rb * 2048 + 512 * j + 16 * lane));
+            tmem_st_32x32b_x4(dst + C::SFB_COL + 8 * j + 4 * rb,
+                              ld_shared_v4(ssfb + rb * C::SFB_ROW_BYTES + 512 * j + 16 * lane));
         }
         tmem_st_wait();
         tc_fence_before();
@@ -1273,6 +1296,14 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       if (lane == 0) mbar_arrive_cluster(leader_bar(&acce_bar));
       acc_phase ^= 1u;
       const float rs = row_ok ? args.xg[row] * args.wg[0] : 0.0f;
+      if constexpr (!C::TMA_STORE) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int col0 = w.n * C::BN + 128 * h + 32 * c;
+          if (row_ok && col0 < args.N) store_output<true>(args, row, col0, rs, r[c]);
+        }
+        continue;
+      }
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
         const int col0 = w.n * C::BN + 128 * h + C::OUT_BOX_COLS * b;
@@ -1299,7 +1330,7 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         }
       }
     }
-    if (lane == 0) bulk_wait_group0();
+    if (C::TMA_STORE && lane == 0) bulk_wait_group0();
   }
 
   // Neither CTA leaves (or frees its TMEM) while the other may still signal
@@ -1415,6 +1446,22 @@ bool make_out_map(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Packed codes [rows, pitch bytes] viewed as [pitch / 128 chunks][rows][128
+// bytes] for 3-D boxes of 128 bytes x box_rows x box_chunks, 128-byte swizzle
+// (each chunk of the box lands as its own swizzled block).  pitch % 128 == 0.
+bool make_chunk_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t pitch, uint32_t box_rows,
+                    uint32_t box_chunks) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc || pitch % 128 != 0) return false;
+  const cuuint64_t dims[3] = {128, rows, pitch / 128};
+  const cuuint64_t strides[2] = {pitch, 128};
+  const cuuint32_t box[3] = {128, box_rows, box_chunks};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Launch arguments shared by both GEMM kernels (BN: tile width).
 GemmArgs make_args(bool fp4, int BN, const uint8_t* xs, const float* xg, const uint8_t* ws, const float* wg,
                    const void* residual, void* Y, int64_t M, int64_t N, int64_t K, void* workspace,
@@ -1463,8 +1510,9 @@ cudaError_t run_fp4(const uint8_t* xq, const uint8_t* xs, const float* xg, const
   return launch_pdl(gemm_fp4_sfw_kernel, dim3(grid), dim3(SfwCfg::THREADS), SfwCfg::SMEM_BYTES, s, ta, tb, a);
 }
 
-// Clusters of gemm_fp4_pair_kernel that fit on the device at once (cached
-// per device; half the SMs when the query fails).
+// Clusters of gemm_fp4_pair_kernel<CH> that fit on the device at once
+// (cached per device; half the SMs when the query fails).
+template <int CH>
 int pair_clusters_resident() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return device_sm_count() / 2;
@@ -1472,10 +1520,10 @@ int pair_clusters_resident() {
   if (dev < 64 && cache[dev]) return cache[dev];
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned int>(device_sm_count()));
-  cfg.blockDim = dim3(PairCfg::THREADS);
-  cfg.dynamicSmemBytes = PairCfg::SMEM_BYTES;
+  cfg.blockDim = dim3(PairCfg<CH>::THREADS);
+  cfg.dynamicSmemBytes = PairCfg<CH>::SMEM_BYTES;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_fp4_pair_kernel, &cfg) != cudaSuccess || n <= 0) {
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_fp4_pair_kernel<CH>, &cfg) != cudaSuccess || n <= 0) {
     cudaGetLastError();
     n = device_sm_count() / 2;
   }
@@ -1483,32 +1531,49 @@ int pair_clusters_resident() {
   return n;
 }
 
-// NVFP4 over CTA pairs: 256 x 256 tiles, direct epilogue through TMA
-// stores.  An output the store map cannot describe (base not 16-byte
-// aligned) runs the single-CTA kernel instead.
+template <int CH>
+cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty, GemmArgs a,
+                        const GemmPlan& plan, cudaStream_t s) {
+  using C = PairCfg<CH>;
+  a.k_tiles = (a.k_steps + C::STEPS - 1) / C::STEPS;
+  cudaError_t e = cudaFuncSetAttribute(gemm_fp4_pair_kernel<CH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  int pairs = pair_clusters_resident<CH>();
+  if (plan.grid / 2 < pairs) pairs = plan.grid / 2;
+  if (a.units < pairs) pairs = a.units;
+  if (pairs < 1) pairs = 1;
+  return launch_pdl(gemm_fp4_pair_kernel<CH>, dim3(static_cast<unsigned int>(2 * pairs)), dim3(C::THREADS),
+                    C::SMEM_BYTES, s, ta, tb, ty, a);
+}
+
+// NVFP4 over CTA pairs: 256 x 256 tiles, direct epilogue.  Rows of whole
+// 128-byte chunks (K % 256 == 0) take two chunks per stage through 3-D
+// boxes; other K one chunk per stage with TMA stores of the output, and an
+// output the store map cannot describe (base not 16-byte aligned) the
+// single-CTA kernel.
 cudaError_t run_fp4_pair(const uint8_t* xq, const uint8_t* xs, const float* xg, const uint8_t* wq, const uint8_t* ws,
                          const float* wg, const void* residual, void* Y, int64_t M, int64_t N, int64_t K,
                          void* workspace, const GemmPlan& plan, long long budget, cudaStream_t s) {
   const int64_t pitch = nvfp4_code_pitch(K);
+  GemmArgs a = make_args(true, PairCfg<1>::BN, xs, xg, ws, wg, residual, Y, M, N, K, nullptr, plan, budget);
+  a.m_tiles = static_cast<int>((M + PairCfg<1>::BM - 1) / PairCfg<1>::BM);
+  a.splits = 1;
+  a.units = a.m_tiles * a.n_tiles;
   CUtensorMap ta, tb, ty;
+  if (K % 256 == 0) {
+    if (!make_chunk_map(&ta, xq, static_cast<uint64_t>(M), static_cast<uint64_t>(pitch), 128, 2) ||
+        !make_chunk_map(&tb, wq, static_cast<uint64_t>(N), static_cast<uint64_t>(pitch), 128, 2))
+      return cudaErrorInvalidValue;
+    ty = tb;  // not read: this variant stores rows directly
+    return launch_pair<2>(ta, tb, ty, a, plan, s);
+  }
   if (!make_out_map(&ty, Y, static_cast<uint64_t>(N), static_cast<uint64_t>(M)))
     return run_fp4(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
   if (!make_map(&ta, xq, static_cast<uint64_t>(pitch), static_cast<uint64_t>(M), static_cast<uint64_t>(pitch), 128) ||
       !make_map(&tb, wq, static_cast<uint64_t>(pitch), static_cast<uint64_t>(N), static_cast<uint64_t>(pitch), 128))
     return cudaErrorInvalidValue;
-  GemmArgs a = make_args(true, PairCfg::BN, xs, xg, ws, wg, residual, Y, M, N, K, nullptr, plan, budget);
-  a.m_tiles = static_cast<int>((M + PairCfg::BM - 1) / PairCfg::BM);
-  a.splits = 1;
-  a.units = a.m_tiles * a.n_tiles;
-  cudaError_t e =
-      cudaFuncSetAttribute(gemm_fp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  int pairs = pair_clusters_resident();
-  if (plan.grid / 2 < pairs) pairs = plan.grid / 2;
-  if (a.units < pairs) pairs = a.units;
-  if (pairs < 1) pairs = 1;
-  return launch_pdl(gemm_fp4_pair_kernel, dim3(static_cast<unsigned int>(2 * pairs)), dim3(PairCfg::THREADS),
-                    PairCfg::SMEM_BYTES, s, ta, tb, ty, a);
+  return launch_pair<1>(ta, tb, ty, a, plan, s);
 }
 
 // FP8 / INT8: gemm_fp8_kernel<BN, I8>, then the ordered split-K reduction
