@@ -1302,31 +1302,31 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
           const int col0 = w.n * C::BN + 128 * h + 32 * c;
           if (row_ok && col0 < args.N) store_output<true>(args, row, col0, rs, r[c]);
         }
-        continue;
-      }
+      } else {
 #pragma unroll
-      for (int b = 0; b < 2; ++b) {
-        const int col0 = w.n * C::BN + 128 * h + C::OUT_BOX_COLS * b;
-        if (col0 >= args.N || row0 >= args.M) continue;  // box wholly outside the output (warp-uniform)
-        if (lane == 0) bulk_wait_group_read0();          // the previous store has read the staging box
-        __syncwarp();
+        for (int b = 0; b < 2; ++b) {
+          const int col0 = w.n * C::BN + 128 * h + C::OUT_BOX_COLS * b;
+          if (col0 >= args.N || row0 >= args.M) continue;  // box wholly outside the output (warp-uniform)
+          if (lane == 0) bulk_wait_group_read0();          // the previous store has read the staging box
+          __syncwarp();
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          if (row_ok) epilogue_values<true>(args, row, col0 + 32 * c, rs, r[2 * b + c]);
-          const float* y = reinterpret_cast<const float*>(r[2 * b + c]);  // rows from M on: clipped by the store
+          for (int c = 0; c < 2; ++c) {
+            if (row_ok) epilogue_values<true>(args, row, col0 + 32 * c, rs, r[2 * b + c]);
+            const float* y = reinterpret_cast<const float*>(r[2 * b + c]);  // rows from M on: clipped by the store
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {  // 16-byte chunk 4c + j of this row, swizzled by row % 8
-            const uint32_t chunk = static_cast<uint32_t>((4 * c + j) ^ (lane & 7));
-            st_shared_v4(box + 128 * lane + 16 * chunk, pack_bf16x2(y[8 * j], y[8 * j + 1]),
-                         pack_bf16x2(y[8 * j + 2], y[8 * j + 3]), pack_bf16x2(y[8 * j + 4], y[8 * j + 5]),
-                         pack_bf16x2(y[8 * j + 6], y[8 * j + 7]));
+            for (int j = 0; j < 4; ++j) {  // 16-byte chunk 4c + j of this row, swizzled by row % 8
+              const uint32_t chunk = static_cast<uint32_t>((4 * c + j) ^ (lane & 7));
+              st_shared_v4(box + 128 * lane + 16 * chunk, pack_bf16x2(y[8 * j], y[8 * j + 1]),
+                           pack_bf16x2(y[8 * j + 2], y[8 * j + 3]), pack_bf16x2(y[8 * j + 4], y[8 * j + 5]),
+                           pack_bf16x2(y[8 * j + 6], y[8 * j + 7]));
+            }
           }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tmY, smem + C::OUT_OFFSET + e * C::OUT_BYTES, col0, row0);
-          bulk_commit_group();
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmY, smem + C::OUT_OFFSET + e * C::OUT_BYTES, col0, row0);
+            bulk_commit_group();
+          }
         }
       }
     }
