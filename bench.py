@@ -733,14 +733,23 @@ def decode_section(vq, data, args, dist_on, device, peaks, world):
     return res
 
 
+GEMM_TIMING = ("gemm_achieved: the four GEMMs back to back over weight copies > L2 (per-launch times, CUDA "
+               "events around the graph); in_step: event nodes around each launch inside the step")
+
+
 def w8a8_section(vq, data, args, dist_on, device, peaks, world, fmt, fused=False):
     fstep = Step(vq, data, M_PREFILL, device, fmt=fmt, fused=fused)
     fms, _, fgem, _ = step_section(vq, fstep, args, dist_on, device, peaks, world)
     fgem_ms = sum(sum(x) for x in fgem) / len(fgem[0])
+    gb2b = gemm_back_to_back(fstep, args, dist_on, device)
+    gb_ms = sum(gb2b.values())
     fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
     out = {"value": world * fstep.flops / (fms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": fms,
-           "gemm_achieved": fstep.flops / (fgem_ms / 1e3) / 1e12, "peak": fp8_peak,
-           "frac": fstep.flops / (fgem_ms / 1e3) / 1e12 / fp8_peak}
+           "gemm_achieved": fstep.flops / (gb_ms / 1e3) / 1e12, "peak": fp8_peak,
+           "frac": fstep.flops / (gb_ms / 1e3) / 1e12 / fp8_peak,
+           "gemm_achieved_in_step": fstep.flops / (fgem_ms / 1e3) / 1e12,
+           "frac_in_step": fstep.flops / (fgem_ms / 1e3) / 1e12 / fp8_peak,
+           "gemm_us": {k: 1e3 * v for k, v in gb2b.items()}, "timing": GEMM_TIMING}
     del fstep
     return out
 
@@ -751,15 +760,20 @@ def fused_section(vq, data, args, dist_on, device, peaks, world):
     step = Step(vq, data, M_PREFILL, device, fused=True)
     ms, pro, gem, _ = step_section(vq, step, args, dist_on, device, peaks, world)
     b2b = prologue_back_to_back(step, args, dist_on, device)
+    gb2b = gemm_back_to_back(step, args, dist_on, device)
     pro_bytes = sum(step.prologue_bytes(L) for L in step.layers)
     gemm_ms = sum(statistics.mean(x) for x in gem)
+    gb_ms = sum(gb2b.values())
     out = {"nvfp4": {
         "value": world * step.flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
-        "gemm_tflops": step.flops / (gemm_ms / 1e3) / 1e12, "gemm_frac": step.flops / (gemm_ms / 1e3) / 1e12 / fp4_peak,
+        "gemm_tflops": step.flops / (gb_ms / 1e3) / 1e12, "gemm_frac": step.flops / (gb_ms / 1e3) / 1e12 / fp4_peak,
+        "gemm_tflops_in_step": step.flops / (gemm_ms / 1e3) / 1e12,
+        "gemm_frac_in_step": step.flops / (gemm_ms / 1e3) / 1e12 / fp4_peak, "timing": GEMM_TIMING,
         "prologue_gbs": pro_bytes / (sum(b2b.values()) / 1e3) / 1e9,
         "prologue_frac": pro_bytes / (sum(b2b.values()) / 1e3) / 1e9 / peaks["hbm_gbs"],
         "per_projection": {L["name"]: {"flags": L["flags"], "residual": L["R"] is not None,
                                        "prologue_us": 1e3 * b2b[L["name"]],
+                                       "gemm_us": 1e3 * gb2b[L["name"]],
                                        "gemm_us_in_step": 1e3 * statistics.mean(gem[i])}
                            for i, L in enumerate(step.layers)},
         "workload": "RMSNorm (gain U(0.5,1.5), eps 1e-6) + block-64 WHT on qkv / gate_up inputs, WHT + residual "

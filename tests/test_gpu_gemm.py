@@ -127,6 +127,38 @@ def test_end_to_end_nvfp4(M, N, K, flags, res):
     check_gemm(Y, Y64, dx, dw, K, residual_f64(R), f"end to end M={M} N={N} K={K} flags={flags}")
 
 
+@pytest.mark.parametrize("M,N,K", [(1024, 2560, 1024), (8, 1024, 3584), (1, 512, 4096)])
+def test_weights_quantized_right_before_linear(M, N, K):
+    """The stream-order contract of vlaq_linear_nvfp4: the GEMM may read wq /
+    ws before its dependency wait, and weights quantized by
+    vlaq_quantize_weight_nvfp4 immediately before it are complete (their
+    codes and scales come from its second-to-last kernel).  Everything is
+    allocated first; then the activation quantizer, the weight quantizer and
+    the GEMM are launched back to back on the stream, nothing in between
+    (CTA pairs, split-K tensor-core path, few-row kernel)."""
+    m = vq()
+    X = si.projection_activations(K, M, 51)
+    W = si.projection_weight(K, N, 51)
+    cx, sx, gx = oracle.quantize_nvfp4(bits(X))
+    cw, sw, gw = oracle.quantize_nvfp4(bits(W), per_tensor=True)
+    dx = oracle.decode_nvfp4(cx, sx, gx, K)
+    dw = oracle.decode_nvfp4(cw, sw, gw, K, per_tensor=True)
+    Y64 = oracle.linear_f64(dx, dw, None)
+    Xd, Wd = X.cuda(), W.cuda()
+    xq, xs, xg = m.alloc_nvfp4(M, K)
+    wq, ws, wg = m.alloc_nvfp4(N, K, per_tensor=True)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    wsp, nb = m.alloc_workspace(M, N, K)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        m.vlaq_quantize_act_nvfp4(Xd, M, K, None, 1e-6, 0, xq, xs, xg)
+        m.vlaq_quantize_weight_nvfp4(Wd, N, K, 0, wq, ws, wg)
+        m.vlaq_linear_nvfp4(xq, xs, xg, wq, ws, wg, None, Y, M, N, K, wsp, nb)
+        torch.cuda.synchronize()
+        m.vlaq_check()
+        check_gemm(Y.float().cpu().numpy(), Y64, dx, dw, K, None, f"weights right before M={M} N={N} K={K}")
+
+
 def test_workspace_is_checked():
     m = vq()
     M, N, K = 8, 512, 4096
