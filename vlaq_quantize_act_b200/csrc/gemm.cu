@@ -449,58 +449,51 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 // allocates 128 registers at entry).
 // Last split of a tile: output = bf16(sum of the splits' fp32 partials, in
 // split order) * g_x[m] g_w + residual.  The tile's valid outputs are spread
-// over `nthreads` threads in 8-column groups; each group's partial loads are
-// issued four splits at a time so they overlap.
+// over `nthreads` threads in 4-column groups (a decode tile of one row still
+// occupies 64 threads), and each thread issues the partial loads of up to
+// kSplitLoads splits at once, so the reduction costs one L2 round trip per
+// kSplitLoads splits.
+constexpr int kSplitLoads = 16;
 __device__ __forceinline__ void splitk_finish_tile(const GemmArgs& a, int m_tile, int n_tile, int bn, int tid,
                                                    int nthreads) {
   const int r0 = m_tile * kBM, c0 = n_tile * bn;
   const int rows = min(kBM, a.M - r0), cols = min(bn, a.N - c0);
-  const int groups = cols >> 3;  // N % 8 == 0
+  const int groups = cols >> 2;  // N % 8 == 0
   const size_t split_stride = static_cast<size_t>(a.M) * a.N;
   for (int item = tid; item < rows * groups; item += nthreads) {
     const int row = r0 + item / groups;
-    const int col = c0 + 8 * (item % groups);
+    const int col = c0 + 4 * (item % groups);
     const float* src = a.partial + static_cast<size_t>(row) * a.N + col;
-    float acc[8];
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    // absent splits of the last batch read as -0, the exact identity of
+    // the addition: the sums equal the plain split-order sums bit for bit
+    const float4 nz = make_float4(-0.0f, -0.0f, -0.0f, -0.0f);
+    for (int sp = 0; sp < a.splits; sp += kSplitLoads) {
+      float4 v[kSplitLoads];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
-    int sp = 0;
-    for (; sp + 4 <= a.splits; sp += 4) {
-      float4 v[4][2];
+      for (int t = 0; t < kSplitLoads; ++t)
+        v[t] = sp + t < a.splits ? __ldcg(reinterpret_cast<const float4*>(src + (sp + t) * split_stride)) : nz;
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const float4* p = reinterpret_cast<const float4*>(src + (sp + t) * split_stride);
-        v[t][0] = __ldcg(p);
-        v[t][1] = __ldcg(p + 1);
+      for (int t = 0; t < kSplitLoads; ++t) {
+        acc[0] += v[t].x;
+        acc[1] += v[t].y;
+        acc[2] += v[t].z;
+        acc[3] += v[t].w;
       }
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        acc[0] += v[t][0].x; acc[1] += v[t][0].y; acc[2] += v[t][0].z; acc[3] += v[t][0].w;
-        acc[4] += v[t][1].x; acc[5] += v[t][1].y; acc[6] += v[t][1].z; acc[7] += v[t][1].w;
-      }
-    }
-    for (; sp < a.splits; ++sp) {
-      const float4* p = reinterpret_cast<const float4*>(src + sp * split_stride);
-      const float4 v0 = __ldcg(p), v1 = __ldcg(p + 1);
-      acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
-      acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
     }
     const float rs = a.xg[row] * a.wg[0];
-    float y[8];
+    float y[4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) y[j] = acc[j] * rs;
+    for (int j = 0; j < 4; ++j) y[j] = acc[j] * rs;
     const size_t o = static_cast<size_t>(row) * a.N + col;
     if (a.residual) {
-      const uint4 rv = __ldg(reinterpret_cast<const uint4*>(a.residual + o));
-      const uint32_t wv[4] = {rv.x, rv.y, rv.z, rv.w};
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        y[2 * t] += __uint_as_float(wv[t] << 16);
-        y[2 * t + 1] += __uint_as_float(wv[t] & 0xFFFF0000u);
-      }
+      const uint2 rv = __ldg(reinterpret_cast<const uint2*>(a.residual + o));
+      y[0] += __uint_as_float(rv.x << 16);
+      y[1] += __uint_as_float(rv.x & 0xFFFF0000u);
+      y[2] += __uint_as_float(rv.y << 16);
+      y[3] += __uint_as_float(rv.y & 0xFFFF0000u);
     }
-    *reinterpret_cast<uint4*>(a.Y + o) = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
-                                                    pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+    *reinterpret_cast<uint2*>(a.Y + o) = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
   }
 }
 
