@@ -1411,6 +1411,271 @@ EncodeTiledFn get_encode_fn() {
 
 // 2-D byte tensor [rows, row_bytes] with the given pitch, box 128 x box_rows,
 // 128-byte swizzle, zero fill out of bounds.
+// 8-bit GEMM over CTA pairs (prefill shapes): FP8 E4M3 (kind::f8f6f4, fp32
+// accumulators) or INT8 (I8: kind::i8, exact s32), 256 x 256 tiles of the
+// paired MMA (tcgen05.mma.cta_group::2) across the two CTAs of a cluster.
+// Without block scales the whole TMEM is accumulator: two 256-column
+// buffers, so the epilogue of one tile runs while the next tile's MMAs
+// accumulate.  CTA r of the pair loads rows [128 r, 128 r + 128) of the A
+// and B tiles, two 128-byte K-chunks (K = 256) per stage through 3-D boxes
+// (K % 256 == 0), and the leader's full barrier completes on both CTAs'
+// bytes.  The leader (even CTA) issues the MMAs and commits each stage to
+// both CTAs' empty barriers; each CTA reads its own 128 accumulator rows and
+// stores them directly (per-row activation scale, per-column weight scale,
+// residual).  Weight tiles of the first stages are loaded before the
+// dependency wait.
+//   warp 0: operand producer (both CTAs); warp 1: TMEM allocator (both) and
+//   MMA issuer (leader); warps 2-9: epilogue, warp e = w - 2 owns TMEM lanes
+//   32 (w % 4) .. + 31 and columns 128 (e / 4) .. + 127.
+template <bool I8>
+struct Fp8PairCfg {
+  static constexpr int BM = 256;
+  static constexpr int BN = 256;
+  static constexpr int CH = 2;
+  static constexpr int CHUNK_BYTES = 128 * 128;
+  static constexpr int A_BYTES = CH * CHUNK_BYTES;
+  static constexpr int B_BYTES = CH * CHUNK_BYTES;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STEPS = 4 * CH;  // MMAs (K = 32) per stage
+  static constexpr int STAGES = 3;
+  static constexpr int ACC_BUFS = 2;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+  static constexpr uint32_t IDESC = (I8 ? (2u << 4) | (1u << 7) | (1u << 10) : (1u << 4)) |
+                                    (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+  static_assert(ACC_BUFS * BN <= kTmemCols, "TMEM budget");
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+template <bool I8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fp8PairCfg<I8>::THREADS, 1)
+gemm_fp8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const GemmArgs args) {
+  using C = Fp8PairCfg<I8>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[C::STAGES];      // leader: operands of both CTAs
+  __shared__ __align__(8) uint64_t empty_bar[C::STAGES];     // stage consumed (leader's commit)
+  __shared__ __align__(8) uint64_t accf_bar[C::ACC_BUFS];    // accumulator complete (leader's commit)
+  __shared__ __align__(8) uint64_t acce_bar[C::ACC_BUFS];    // leader: both CTAs' accumulators read
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t s_tmem_base;
+  __shared__ volatile int s_abort;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int pairs = static_cast<int>(gridDim.x >> 1);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < C::ACC_BUFS; ++i) {
+      mbar_init(&accf_bar[i], 1);
+      mbar_init(&acce_bar[i], 2 * C::EPI_WARPS);
+    }
+    mbar_init(&drain_bar, 1);
+    s_abort = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&s_tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();  // both CTAs' barriers are initialised before either CTA signals the other's
+  tc_fence_after();
+  const uint32_t tmem = s_tmem_base;
+  const uint32_t peer_abort = mapa_shared(smem_u32(const_cast<int*>(&s_abort)), rank ^ 1u);
+  auto leader_bar = [&](uint64_t* bar) { return mapa_shared(smem_u32(bar), 0u); };
+  auto stage_steps = [&](int kt) { return min(C::STEPS, args.k_steps - C::STEPS * kt); };
+  auto issue_weights = [&](int stage, const Unit& w, int kt) {
+    tma_load_3d_pair(smem + stage * C::STAGE_BYTES + C::A_BYTES, &tmB, leader_bar(&full_bar[stage]), 0,
+                     w.n * C::BN + 128 * static_cast<int>(rank), kt * C::CH);
+  };
+  auto issue_acts = [&](int stage, const Unit& w, int kt) {
+    tma_load_3d_pair(smem + stage * C::STAGE_BYTES, &tmA, leader_bar(&full_bar[stage]), 0,
+                     w.m * C::BM + 128 * static_cast<int>(rank), kt * C::CH);
+  };
+
+  // Weights do not depend on the previous kernel on the stream: the first
+  // stages' weight tiles stream in before the dependency wait.
+  int pre = 0;
+  uint32_t armed = 0;
+  if (warp == 0 && lane == 0) {
+    for (int u = pair; u < args.units && pre < C::STAGES; u += pairs) {
+      const Unit w = decode_unit(args, u);
+      for (int kt = w.kt0; kt < w.kt1 && pre < C::STAGES; ++kt, ++pre) {
+        if (rank == 0) mbar_arrive_expect_tx(&full_bar[pre], 2 * C::STAGE_BYTES);
+        armed |= 1u << pre;
+        issue_weights(pre, w, kt);
+      }
+    }
+  }
+  griddep_wait();
+  griddep_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------- operand producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed_phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int u = pair; u < args.units && ok; u += pairs) {
+        const Unit w = decode_unit(args, u);
+        for (int kt = w.kt0; kt < w.kt1; ++kt, ++it) {
+          if (it >= pre) {
+            if (!pair_wait(&empty_bar[stage], phase ^ 1u, args.budget, &s_abort, peer_abort)) {
+              ok = false;
+              break;
+            }
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * C::STAGE_BYTES);
+            armed |= 1u << stage;
+            armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+            issue_weights(stage, w, kt);
+          }
+          issue_acts(stage, w, kt);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (ok) {
+        // every stage released: the leader's last commits to this CTA have landed
+        for (int i = 0; i < C::STAGES && ok; ++i) {
+          ok = pair_wait(&empty_bar[stage], phase ^ 1u, args.budget, &s_abort, peer_abort);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      } else if (rank == 0) {
+        for (int i = 0; i < C::STAGES; ++i)
+          if (armed & (1u << i)) {
+            const long long t0 = clock64();
+            while (!mbar_try_wait(&full_bar[i], (armed_phase >> i) & 1u) && clock64() - t0 < args.budget) {
+            }
+          }
+      } else {
+        // the peer cannot observe the leader's barriers: give its copies in
+        // flight time to land before the pair's final barrier
+        const long long t0 = clock64();
+        while (clock64() - t0 < (1ll << 21)) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (leader)
+    if (lane == 0 && rank == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int u = pair; u < args.units && ok; u += pairs) {
+        const Unit w = decode_unit(args, u);
+        if (!pair_wait(&acce_bar[acc], acc_phase ^ 1u, args.budget, &s_abort, peer_abort)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * C::BN);
+        for (int kt = w.kt0; kt < w.kt1; ++kt) {
+          if (!pair_wait(&full_bar[stage], phase, args.budget, &s_abort, peer_abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES), b0 = a0 + C::A_BYTES;
+          const int steps = stage_steps(kt);
+          for (int j = 0; j < steps; ++j) {
+            const uint32_t off = (j >> 2) * C::CHUNK_BYTES + 32 * (j & 3);  // chunk, then 32 K within it
+            const uint64_t ad = sdesc_kmajor_sw128(a0 + off), bd = sdesc_kmajor_sw128(b0 + off);
+            const uint32_t accum = (kt > w.kt0 || j > 0) ? 1u : 0u;
+            if constexpr (I8)
+              mma_i8_pair(d_tmem, ad, bd, C::IDESC, accum);
+            else
+              mma_f8f6f4_pair(d_tmem, ad, bd, C::IDESC, accum);
+          }
+          umma_commit_pair(&empty_bar[stage], 0x3);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(&accf_bar[acc], 0x3);
+        if (++acc == C::ACC_BUFS) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      umma_commit_pair(&drain_bar, 0x1);
+      const long long t0 = clock64();
+      while (!mbar_try_wait(&drain_bar, 0) && clock64() - t0 < 4 * args.budget + 1000000) {
+      }
+    }
+  } else {
+    // ------------------------------------------------- epilogue (both CTAs)
+    const int e = warp - 2;
+    const int q = warp & 3;
+    const int h = e >> 2;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = pair; u < args.units; u += pairs) {
+      const Unit w = decode_unit(args, u);
+      if (!pair_wait(&accf_bar[acc], acc_phase, args.budget, &s_abort, peer_abort)) break;
+      tc_fence_after();
+      const int row = w.m * C::BM + 128 * static_cast<int>(rank) + 32 * q + lane;
+      const bool row_ok = row < args.M;
+      const uint32_t tbase =
+          tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * C::BN + 128 * h);
+      __syncwarp();
+      const float rs = row_ok ? args.xg[row] : 0.0f;
+      // 64 columns at a time (the other accumulator buffer keeps the MMAs
+      // busy meanwhile); the buffer is handed back after the last load
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        uint32_t r[2][32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) tmem_ld_32x32b_x32(tbase + 64 * g + 32 * c, r[c]);
+        tmem_ld_wait();
+        if (g == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(leader_bar(&acce_bar[acc]));
+        }
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int col0 = w.n * C::BN + 128 * h + 64 * g + 32 * c;
+          if (row_ok && col0 < args.N) store_output<false, I8>(args, row, col0, rs, r[c]);
+        }
+      }
+      if (++acc == C::ACC_BUFS) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  // Neither CTA leaves (or frees its TMEM) while the other may still signal
+  // it or the paired MMAs may still touch its shared memory or TMEM.
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
 bool make_map(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows, uint64_t pitch,
               uint32_t box_rows) {
   EncodeTiledFn enc = get_encode_fn();
@@ -1569,6 +1834,53 @@ cudaError_t run_fp4_pair(const uint8_t* xq, const uint8_t* xs, const float* xg, 
   return launch_pair<1>(ta, tb, ty, a, plan, s);
 }
 
+// Clusters of gemm_fp8_pair_kernel<I8> that fit on the device at once
+// (cached per device; half the SMs when the query fails).
+template <bool I8>
+int fp8_pair_clusters_resident() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return device_sm_count() / 2;
+  static int cache[64] = {0};
+  if (dev < 64 && cache[dev]) return cache[dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned int>(device_sm_count()));
+  cfg.blockDim = dim3(Fp8PairCfg<I8>::THREADS);
+  cfg.dynamicSmemBytes = Fp8PairCfg<I8>::SMEM_BYTES;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_fp8_pair_kernel<I8>, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = device_sm_count() / 2;
+  }
+  if (dev < 64) cache[dev] = n;
+  return n;
+}
+
+// FP8 / INT8 over CTA pairs: 256 x 256 tiles, two K-chunks per stage (K %
+// 256 == 0), direct epilogue, no split.
+template <bool I8>
+cudaError_t run_fp8_pair(const uint8_t* xq, const float* xg, const uint8_t* wq, const float* wg,
+                         const void* residual, void* Y, int64_t M, int64_t N, int64_t K, const GemmPlan& plan,
+                         long long budget, cudaStream_t s) {
+  using C = Fp8PairCfg<I8>;
+  CUtensorMap ta, tb;
+  if (!make_chunk_map(&ta, xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K), 128, C::CH) ||
+      !make_chunk_map(&tb, wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K), 128, C::CH))
+    return cudaErrorInvalidValue;
+  GemmArgs a = make_args(false, C::BN, nullptr, xg, nullptr, wg, residual, Y, M, N, K, nullptr, plan, budget);
+  a.m_tiles = static_cast<int>((M + C::BM - 1) / C::BM);
+  a.splits = 1;
+  a.units = a.m_tiles * a.n_tiles;
+  a.k_tiles = (a.k_steps + C::STEPS - 1) / C::STEPS;
+  auto kern = gemm_fp8_pair_kernel<I8>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  int pairs = fp8_pair_clusters_resident<I8>();
+  if (plan.grid / 2 < pairs) pairs = plan.grid / 2;
+  if (a.units < pairs) pairs = a.units;
+  if (pairs < 1) pairs = 1;
+  return launch_pdl(kern, dim3(static_cast<unsigned int>(2 * pairs)), dim3(C::THREADS), C::SMEM_BYTES, s, ta, tb, a);
+}
+
 // FP8 / INT8: gemm_fp8_kernel<BN, I8>, then the ordered split-K reduction
 // when split.
 template <int BN, bool I8>
@@ -1645,6 +1957,14 @@ GemmPlan plan_gemm(bool fp4, int64_t M, int64_t N, int64_t K, int num_sms) {
     p.splits = 1;
     p.grid = static_cast<int>(tiles256 < num_sms ? tiles256 : num_sms);
     p.ws_bytes = 0;
+    // more than 128 rows and rows of whole 256-byte K-chunks: 256 x 256
+    // tiles over CTA pairs
+    if (M > kBM && K % 256 == 0) {
+      const int64_t pair_units = ((M + 255) / 256) * ((N + 255) / 256);
+      const int64_t pairs = num_sms / 2;
+      p.pair = true;
+      p.grid = static_cast<int>(2 * (pair_units < pairs ? pair_units : pairs));
+    }
     return p;
   }
   // Few output tiles (decode): narrow tiles and split-K over the SMs.
@@ -1672,6 +1992,7 @@ cudaError_t launch_linear(bool fp4, const uint8_t* xq, const uint8_t* xs, const 
   if (fp4 && plan.pair)
     return run_fp4_pair(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
   if (fp4) return run_fp4(xq, xs, xg, wq, ws, wg, residual, Y, M, N, K, workspace, plan, budget, s);
+  if (plan.pair) return run_fp8_pair<false>(xq, xg, wq, wg, residual, Y, M, N, K, plan, budget, s);
   if (plan.bn == 256) return run_fp8<256, false>(xq, xg, wq, wg, residual, Y, M, N, K, workspace, plan, budget, s);
   return run_fp8<128, false>(xq, xg, wq, wg, residual, Y, M, N, K, workspace, plan, budget, s);
 }
@@ -1681,6 +2002,7 @@ cudaError_t launch_linear_int8(const int8_t* xq, const float* s_x, const int8_t*
                                const GemmPlan& plan, long long budget, cudaStream_t s) {
   const uint8_t* x8 = reinterpret_cast<const uint8_t*>(xq);
   const uint8_t* w8 = reinterpret_cast<const uint8_t*>(wq);
+  if (plan.pair) return run_fp8_pair<true>(x8, s_x, w8, s_w, residual, Y, M, N, K, plan, budget, s);
   if (plan.bn == 256) return run_fp8<256, true>(x8, s_x, w8, s_w, residual, Y, M, N, K, workspace, plan, budget, s);
   return run_fp8<128, true>(x8, s_x, w8, s_w, residual, Y, M, N, K, workspace, plan, budget, s);
 }
