@@ -117,9 +117,19 @@ def test_fused_prologue_m1024(name, flags, residual):
 
 @pytest.mark.parametrize("name,flags,residual", [("qkv", 3, False), ("down", 2, True)])
 def test_fused_fp8_m1024(name, flags, residual):
+    _run_fp8(name, 1024, flags, residual)
+
+
+def test_fp8_m4580():
+    """The FP8 GEMM over CTA pairs at M = 4580 on the o shape: 18 x 14 tiles
+    of 256 x 256 on 74 clusters (several tiles per cluster through both
+    accumulator buffers, a ragged last row tile), with the residual."""
+    _run_fp8("o", 4580, 0, True)
+
+
+def _run_fp8(name, M, flags, residual):
     m = vq()
     K, N, seed = si.PROJECTIONS[name]
-    M = 1024
     W = si.projection_weight(K, N, seed)
     X = si.projection_activations(K, M, seed)
     gam = si.norm_gain(K, seed)

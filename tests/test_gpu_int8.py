@@ -144,6 +144,38 @@ def test_end_to_end_int8(M, N, K, flags, res):
     assert_bits_equal(Y.cpu().view(torch.int16).numpy().view(np.uint16), want, f"int8 e2e {M}x{N}x{K}")
 
 
+def test_linear_int8_m4580_sampled_rows():
+    """The INT8 GEMM over CTA pairs at M = 4580, o shape (3584 x 3584) with
+    the residual: 18 x 14 tiles of 256 x 256 on 74 clusters, so clusters run
+    several tiles through both accumulator buffers and the last row tile is
+    ragged (4580 = 17 * 256 + 228); outputs bit-exact on sampled rows, one
+    in every 128-row block."""
+    m = vq()
+    M, N, K = 4580, 3584, 3584
+    X = si.projection_activations(K, M, 57)
+    W = si.projection_weight(K, N, 57)
+    R = si.residual(M, N, 57)
+    xq, sx = m.alloc_int8(M, K)
+    wq, sw = m.alloc_int8(N, K)
+    m.vlaq_quantize_weight_int8(W.cuda(), N, K, 0, wq, sw)
+    m.vlaq_quantize_act_int8(X.cuda(), M, K, None, 1e-6, 0, xq, sx)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    wsp, nb = m.alloc_workspace(M, N, K)
+    m.vlaq_linear_int8(xq, sx, wq, sw, R.cuda(), Y, M, N, K, wsp, nb)
+    torch.cuda.synchronize()
+    m.vlaq_check()
+    rng = np.random.default_rng(58)
+    rows = {0, M - 1} | {int(t + rng.integers(0, min(128, M - t))) for t in range(0, M, 128)}
+    rows = np.array(sorted(rows))
+    cx, rsx = oracle.quantize_int8(bits(X)[rows])
+    assert np.array_equal(xq.cpu().numpy()[rows], cx)
+    cw, rsw = oracle.quantize_int8(bits(W))
+    assert np.array_equal(wq.cpu().numpy(), cw)
+    want, _ = oracle.linear_int8(cx, rsx, cw, rsw, bits(R)[rows])
+    got = Y.cpu().view(torch.int16).numpy().view(np.uint16)[rows]
+    assert_bits_equal(got, want, "int8 o M=4580 sampled rows")
+
+
 def test_linear_int8_full_size_sampled_rows():
     """gate_up at the full prefill size (1024 x 37888 x 3584): GPU quantizers
     and GEMM, outputs bit-exact on sampled rows."""
