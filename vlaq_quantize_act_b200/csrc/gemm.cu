@@ -1440,7 +1440,8 @@ struct Fp8PairCfg {
   static constexpr int STAGES = 3;
   static constexpr int ACC_BUFS = 2;
   static constexpr int EPI_WARPS = 8;
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int PRODUCERS = STAGES;  // one producer warp per stage slot
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS + 32 * (PRODUCERS - 1);
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
   static constexpr uint32_t IDESC = (I8 ? (2u << 4) | (1u << 7) | (1u << 10) : (1u << 4)) |
                                     (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
@@ -1507,67 +1508,63 @@ gemm_fp8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                      w.m * C::BM + 128 * static_cast<int>(rank), kt * C::CH);
   };
 
-  // Weights do not depend on the previous kernel on the stream: the first
-  // stages' weight tiles stream in before the dependency wait.
-  int pre = 0;
-  uint32_t armed = 0;
-  if (warp == 0 && lane == 0) {
-    for (int u = pair; u < args.units && pre < C::STAGES; u += pairs) {
+  // Producer p (warp 0, then warps 2 + EPI_WARPS ...) owns stage slot p: it
+  // issues the loads of stages p, p + STAGES, p + 2 STAGES, ... so that
+  // several threads keep TMA copies in flight.  Weights do not depend on the
+  // previous kernel on the stream: each producer's first weight tile
+  // streams in before the dependency wait.
+  const int prod = warp == 0 ? 0 : (warp >= 2 + C::EPI_WARPS ? warp - (1 + C::EPI_WARPS) : -1);
+  bool armed = false;
+  uint32_t armed_phase = 0;
+  if (prod >= 0 && lane == 0) {
+    int it = 0;
+    for (int u = pair; u < args.units && it <= prod; u += pairs) {
       const Unit w = decode_unit(args, u);
-      for (int kt = w.kt0; kt < w.kt1 && pre < C::STAGES; ++kt, ++pre) {
-        if (rank == 0) mbar_arrive_expect_tx(&full_bar[pre], 2 * C::STAGE_BYTES);
-        armed |= 1u << pre;
-        issue_weights(pre, w, kt);
+      for (int kt = w.kt0; kt < w.kt1 && it <= prod; ++kt, ++it) {
+        if (it != prod) continue;
+        if (rank == 0) mbar_arrive_expect_tx(&full_bar[prod], 2 * C::STAGE_BYTES);
+        armed = true;
+        issue_weights(prod, w, kt);
       }
     }
   }
   griddep_wait();
   griddep_launch_dependents();
 
-  if (warp == 0) {
-    // ------------------------------------------- operand producer (both CTAs)
+  if (prod >= 0) {
+    // ------------------------------------------- operand producers (both CTAs)
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t armed_phase = 0;
-      int it = 0;
+      int it = 0, uses = 0;
       bool ok = true;
       for (int u = pair; u < args.units && ok; u += pairs) {
         const Unit w = decode_unit(args, u);
         for (int kt = w.kt0; kt < w.kt1; ++kt, ++it) {
-          if (it >= pre) {
-            if (!pair_wait(&empty_bar[stage], phase ^ 1u, args.budget, &s_abort, peer_abort)) {
+          if (it % C::STAGES != prod) continue;
+          const uint32_t phase = static_cast<uint32_t>(uses) & 1u;
+          if (it >= C::STAGES) {
+            if (!pair_wait(&empty_bar[prod], phase ^ 1u, args.budget, &s_abort, peer_abort)) {
               ok = false;
               break;
             }
-            if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * C::STAGE_BYTES);
-            armed |= 1u << stage;
-            armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
-            issue_weights(stage, w, kt);
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[prod], 2 * C::STAGE_BYTES);
+            armed = true;
+            armed_phase = phase;
+            issue_weights(prod, w, kt);
           }
-          issue_acts(stage, w, kt);
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
+          issue_acts(prod, w, kt);
+          ++uses;
         }
       }
       if (ok) {
-        // every stage released: the leader's last commits to this CTA have landed
-        for (int i = 0; i < C::STAGES && ok; ++i) {
-          ok = pair_wait(&empty_bar[stage], phase ^ 1u, args.budget, &s_abort, peer_abort);
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
+        // the slot released after its last use: the leader's last commit to
+        // this CTA has landed
+        if (uses > 0) pair_wait(&empty_bar[prod], (static_cast<uint32_t>(uses) & 1u) ^ 1u, args.budget, &s_abort, peer_abort);
+      } else if (rank == 0) {
+        if (armed) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(&full_bar[prod], armed_phase) && clock64() - t0 < args.budget) {
           }
         }
-      } else if (rank == 0) {
-        for (int i = 0; i < C::STAGES; ++i)
-          if (armed & (1u << i)) {
-            const long long t0 = clock64();
-            while (!mbar_try_wait(&full_bar[i], (armed_phase >> i) & 1u) && clock64() - t0 < args.budget) {
-            }
-          }
       } else {
         // the peer cannot observe the leader's barriers: give its copies in
         // flight time to land before the pair's final barrier
@@ -1622,7 +1619,7 @@ gemm_fp8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       while (!mbar_try_wait(&drain_bar, 0) && clock64() - t0 < 4 * args.budget + 1000000) {
       }
     }
-  } else {
+  } else if (warp >= 2) {
     // ------------------------------------------------- epilogue (both CTAs)
     const int e = warp - 2;
     const int q = warp & 3;
