@@ -204,9 +204,9 @@ def test_linear_nvfp4_wide_tiles_vs_oracle(M, N, K, res):
 
 # the first two wide cases, then 256 x 256 tiles over CTA pairs (more than
 # 128 rows, enough tiles, K % 256 == 0): ragged M with two tiles per
-# cluster, ragged N with K = 3 stages, K = 1 stage
+# cluster, ragged N with K = 3 stages, K = 1 stage, 200 rows in one tile
 @pytest.mark.parametrize("M,N,K,res", WIDE_CASES[:2] + [(300, 9728, 512, True), (1000, 4104, 768, False),
-                                                        (512, 19200, 256, True)])
+                                                        (512, 19200, 256, True), (200, 19200, 256, False)])
 def test_linear_fp8_wide_tiles_vs_oracle(M, N, K, res):
     X = si.projection_activations(K, M, 33)
     W = si.projection_weight(K, N, 33)

@@ -87,11 +87,13 @@ def test_int8_ties_and_edge_rows():
 # decode rows (split-K over the SMs), both tile widths, the projection
 # shapes; then 256 x 256 tiles over CTA pairs (more than 128 rows, enough
 # tiles, K % 256 == 0): one tile per cluster, ragged M with two tiles per
-# cluster (both accumulator buffers), ragged N with K = 3 stages, K = 1 stage
+# cluster (both accumulator buffers), ragged N with K = 3 stages, K = 1 stage,
+# and 200 rows (one 256-row tile, the second CTA's 128 rows partly past M)
 INT8_GEMMS = [(16, 128, 256, False), (300, 392, 1024, True), (129, 136, 208, False), (1, 512, 4096, True),
               (8, 256, 2048, False), (257, 264, 3584, False), (1, 3584, 18944, True), (4, 4608, 3584, False),
               (1024, 512, 3584, True), (33, 8, 48, True),
-              (1024, 2560, 1024, True), (300, 9728, 512, False), (1000, 4104, 768, True), (512, 19200, 256, False)]
+              (1024, 2560, 1024, True), (300, 9728, 512, False), (1000, 4104, 768, True), (512, 19200, 256, False),
+              (200, 19200, 256, True)]
 
 
 @pytest.mark.parametrize("M,N,K,res", INT8_GEMMS)
