@@ -22,7 +22,9 @@
 //   gemm_fp8_kernel<BN, I8>  FP8 E4M3 (kind::f8f6f4, fp32 accumulators) or
 //                        INT8 (kind::i8, s32), 128 x 256 or 128 x 128 tiles
 //                        (double-buffered accumulator); split-K partials are
-//                        added by splitk_reduce_kernel in fixed order.
+//                        added by splitk_reduce_kernel in fixed order;
+//   gemm_fp8_pair_kernel<I8>  FP8 / INT8, 256 x 256 tiles over CTA pairs
+//                        with two accumulators; prefill shapes.
 // Epilogues: tcgen05.ld of the accumulator, scale, residual add, bf16 round,
 // global stores.
 //
@@ -1424,9 +1426,10 @@ EncodeTiledFn get_encode_fn() {
 // stores them directly (per-row activation scale, per-column weight scale,
 // residual).  Weight tiles of the first stages are loaded before the
 // dependency wait.
-//   warp 0: operand producer (both CTAs); warp 1: TMEM allocator (both) and
-//   MMA issuer (leader); warps 2-9: epilogue, warp e = w - 2 owns TMEM lanes
-//   32 (w % 4) .. + 31 and columns 128 (e / 4) .. + 127.
+//   warps 0, 10, 11: operand producers (both CTAs), one per stage slot;
+//   warp 1: TMEM allocator (both) and MMA issuer (leader); warps 2-9:
+//   epilogue, warp e = w - 2 owns TMEM lanes 32 (w % 4) .. + 31 and
+//   columns 128 (e / 4) .. + 127.
 template <bool I8>
 struct Fp8PairCfg {
   static constexpr int BM = 256;
