@@ -193,6 +193,9 @@ class Step:
         self.layers = []
         for name in PROJ:
             K, N, X, W = data[name]
+            # the library reads M rows of X through a raw pointer
+            if X.shape[0] < M or X.shape[1] != K:
+                raise ValueError(f"{name}: X is {tuple(X.shape)}, the step needs at least {M} x {K}")
             case = FUSED[name]
             flags = (3 if case.rmsnorm else 2) if fused else 0
             wflags = flags & 2
