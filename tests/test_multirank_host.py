@@ -53,6 +53,16 @@ def test_per_rank_inputs_differ_but_share_weights():
         assert not torch.equal(a[name][2], b[name][2])      # X
 
 
+def test_step_refuses_activations_shorter_than_m():
+    """The library reads M rows of X through a raw pointer, so the bench step
+    checks the host tensor before anything is allocated or launched."""
+    import pytest
+    import bench
+    data = bench.make_inputs(16, "cpu")
+    with pytest.raises(ValueError, match="needs at least 32"):
+        bench.Step(None, data, 32, "cpu")
+
+
 def test_reference_arm_under_torchrun_two_ranks():
     port = _free_port()
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
