@@ -178,11 +178,13 @@ def test_linear_int8_m4580_sampled_rows():
     assert_bits_equal(got, want, "int8 o M=4580 sampled rows")
 
 
-def test_linear_int8_full_size_sampled_rows():
-    """gate_up at the full prefill size (1024 x 37888 x 3584): GPU quantizers
-    and GEMM, outputs bit-exact on sampled rows."""
+@pytest.mark.parametrize("N,K", [(37888, 3584), (3584, 18944)])
+def test_linear_int8_full_size_sampled_rows(N, K):
+    """gate_up (1024 x 37888 x 3584) and down (1024 x 3584 x 18944, 37 stages
+    per tile) at the full prefill size: GPU quantizers and GEMM over CTA
+    pairs, outputs bit-exact on sampled rows."""
     m = vq()
-    M, N, K = 1024, 37888, 3584
+    M = 1024
     X = si.projection_activations(K, M, 55)
     W = si.projection_weight(K, N, 55)
     xq, sx = m.alloc_int8(M, K)
@@ -202,4 +204,4 @@ def test_linear_int8_full_size_sampled_rows():
                                                                    rsw.view(np.uint32))
     want, _ = oracle.linear_int8(cx, rsx, cw, rsw)
     got = Y.cpu().view(torch.int16).numpy().view(np.uint16)[rows]
-    assert_bits_equal(got, want, "int8 gate_up sampled rows")
+    assert_bits_equal(got, want, f"int8 {M}x{N}x{K} sampled rows")
