@@ -57,6 +57,12 @@ struct RowCfg {
   // kept transformed values of the fused variants: per warp BPL x 16 fp32
   // per lane
   static constexpr int kCacheBytesPerWarp = BPL * 16 * 4 * 32;
+  // rows of up to 4096 elements: seven CTAs per SM (at most 72 registers),
+  // so that the 1036 resident CTAs hold every row of a 1024-token input
+  // (measured: the fused smoothing variant at 80 registers, six CTAs per SM,
+  // ran 6% slower).  The untransformed static-scale variant stays below 72
+  // registers without the bound and ran 4% slower under it.
+  static constexpr int min_blocks(bool bounded) { return (W == 4 && BPL == 2 && bounded) ? 7 : 1; }
 };
 
 __device__ __forceinline__ void unpack_bf16x8(const uint4& q, float* v) {
@@ -183,29 +189,52 @@ struct RowArgs {
 // each, element 16 (lane % 4) + j): stages h = 1, 2, 4, 8 inside the lane,
 // h = 16, 32 across lanes (xor 1, 2), then x 1/8 (exact) -- the stages of the
 // sequential butterfly in the same order.  Executed by the whole warp.
+// Stages h >= 2 run two butterflies per packed fp32x2 instruction (each lane
+// rounded once, so the values are those of the scalar steps): a + b, and
+// a - b as fma(b, -1, a), a single rounding of the same exact difference
+// (signed zeros included).  Across lanes the new value is p + s v with s = -1
+// in the upper lane and +1 in the lower one, again one fused multiply-add.
 __device__ __forceinline__ void wht64_lanes(float* v, int lane) {
 #pragma unroll
-  for (int h = 1; h < 16; h <<= 1) {
+  for (int i = 0; i < 16; i += 2) {
+    const float a = v[i], b = v[i + 1];
+    v[i] = __fadd_rn(a, b);
+    v[i + 1] = __fsub_rn(a, b);
+  }
+  const float2 m1 = make_float2(-1.0f, -1.0f);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
+  for (int h = 2; h < 16; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
       if ((i & h) == 0) {
-        const float a = v[i], b = v[i + h];
-        v[i] = __fadd_rn(a, b);
-        v[i + h] = __fsub_rn(a, b);
+        const float2 a = make_float2(v[i], v[i + 1]), b = make_float2(v[i + h], v[i + h + 1]);
+        const float2 sum = __fadd2_rn(a, b), dif = __ffma2_rn(b, m1, a);
+        v[i] = sum.x;
+        v[i + 1] = sum.y;
+        v[i + h] = dif.x;
+        v[i + h + 1] = dif.y;
       }
     }
   }
 #pragma unroll
   for (int x = 1; x < 4; x <<= 1) {
-    const bool upper = (lane & x) != 0;
+    const float sg = (lane & x) != 0 ? -1.0f : 1.0f;
+    const float2 s2 = make_float2(sg, sg);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float p = __shfl_xor_sync(0xffffffffu, v[i], x);
-      v[i] = upper ? __fsub_rn(p, v[i]) : __fadd_rn(v[i], p);
+    for (int i = 0; i < 16; i += 2) {
+      const float2 p = make_float2(__shfl_xor_sync(0xffffffffu, v[i], x), __shfl_xor_sync(0xffffffffu, v[i + 1], x));
+      const float2 r = __ffma2_rn(make_float2(v[i], v[i + 1]), s2, p);
+      v[i] = r.x;
+      v[i + 1] = r.y;
     }
   }
+  const float2 e8 = make_float2(0.125f, 0.125f);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], 0.125f);
+  for (int i = 0; i < 16; i += 2) {
+    const float2 r = __fmul2_rn(make_float2(v[i], v[i + 1]), e8);
+    v[i] = r.x;
+    v[i + 1] = r.y;
+  }
 }
 
 // y_k / a_k or y_k * a_k for the 16 channels of block q (smoothing).
@@ -281,7 +310,9 @@ __device__ __forceinline__ float rms_factor_row(const uint4* x4, int K, float ep
 // (per-channel smoothing), W warps per row.  Row group k of the grid takes
 // rows k, k + groups, ... (one row per group at the workload sizes).
 template <int FMT, int MODE, bool NORM, bool WHT, bool SMOOTH, int W, int BPL>
-__global__ void __launch_bounds__(RowCfg<W, BPL>::kThreads) quant_rows_kernel(const RowArgs a) {
+__global__ void __launch_bounds__(RowCfg<W, BPL>::kThreads,
+                                  RowCfg<W, BPL>::min_blocks(NORM || WHT || SMOOTH || MODE != kStatic))
+    quant_rows_kernel(const RowArgs a) {
   using C = RowCfg<W, BPL>;
   constexpr bool KEEP = NORM || WHT || SMOOTH;  // transformed values kept in shared memory
   // dynamic shared memory: [kept values][row copy]
