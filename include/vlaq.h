@@ -212,8 +212,8 @@ VLAQ_API vlaq_status vlaq_scales_to_rowmajor(const uint8_t* in, uint8_t* out, in
 
 /* Bytes of workspace vlaq_linear_nvfp4 / _fp8 / _int8 need for the given
  * shape on the current device (0 when the shape runs without split-K).  The
- * workspace's first 1024 bytes hold vlaq_linear_nvfp4's per-tile arrival
- * counters, the per-split partial sums (fp32, s32 for INT8) follow.  The counters must be
+ * workspace's first 1024 bytes hold the per-tile arrival counters of
+ * split-K calls, the per-split partial sums (fp32, s32 for INT8) follow.  The counters must be
  * zero when a call starts: zero the workspace once after allocating it;
  * every call (of any shape, NVFP4 or FP8) leaves them zero again, so nothing
  * is cleared between calls.  After vlaq_check reports VLAQ_ERR_TIMEOUT, zero

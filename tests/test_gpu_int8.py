@@ -108,6 +108,33 @@ def test_linear_int8_bit_exact(M, N, K, res):
     assert_bits_equal(got, want, f"int8 GEMM {M}x{N}x{K}")
 
 
+def test_int8_split_workspace_reused_across_calls_and_shapes():
+    """The 8-bit split-K tile counters return to zero after every call: one
+    zeroed workspace serves repeated INT8 calls of shapes with different
+    split counts, every output bit-exact (a counter left non-zero would keep
+    a tile's last split from recognising itself)."""
+    m = vq()
+    shapes = [(5, 512, 4096), (8, 1024, 3584), (6, 256, 2048)]
+    need = max(m.vlaq_linear_workspace_bytes(*s) for s in shapes)
+    assert all(m.vlaq_linear_workspace_bytes(*s) > 0 for s in shapes)  # all three split K
+    wsp = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    cases = {}
+    for (M, N, K) in shapes:
+        X = si.projection_activations(K, M, 59)
+        W = si.projection_weight(K, N, 59)
+        cx, sx = oracle.quantize_int8(bits(X))
+        cw, sw = oracle.quantize_int8(bits(W))
+        want, _ = oracle.linear_int8(cx, sx, cw, sw)
+        cases[(M, N, K)] = ((to_dev(cx), to_dev(sx), to_dev(cw), to_dev(sw)), want)
+    for rep in range(3):
+        for (M, N, K), (dev, want) in cases.items():
+            Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+            m.vlaq_linear_int8(*dev, None, Y, M, N, K, wsp, need)
+            torch.cuda.synchronize()
+            m.vlaq_check()
+            assert_bits_equal(Y.cpu().view(torch.int16).numpy().view(np.uint16), want, f"rep {rep} {M}x{N}x{K}")
+
+
 def test_linear_int8_extreme_sums():
     """Every product +-127^2 at the largest K: |acc| = K 127^2 < 2^31, where
     fp32(acc) rounds (acc > 2^24)."""

@@ -21,8 +21,8 @@
 //                        half of the weight tile; prefill shapes;
 //   gemm_fp8_kernel<BN, I8>  FP8 E4M3 (kind::f8f6f4, fp32 accumulators) or
 //                        INT8 (kind::i8, s32), 128 x 256 or 128 x 128 tiles
-//                        (double-buffered accumulator); split-K partials are
-//                        added by splitk_reduce_kernel in fixed order;
+//                        (double-buffered accumulator); split-K (decode
+//                        shapes) reduced in-kernel by the last split;
 //   gemm_fp8_pair_kernel<I8>  FP8 / INT8, 256 x 256 tiles over CTA pairs
 //                        with two accumulators; prefill shapes.
 // Epilogues: tcgen05.ld of the accumulator, scale, residual add, bf16 round,
@@ -232,10 +232,85 @@ __device__ __forceinline__ void store_output(const GemmArgs& a, int row, int col
   }
 }
 
+// Barrier `id` over the first `n` threads' warps that reach it (n a
+// multiple of 32); id 0 is __syncthreads.
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Last split of an 8-bit tile: the splits' partials summed in split order
+// (INT8: exact s32 sums; FP8: fp32 from 0, absent splits of a batch read as
+// -0, the exact identity of the addition), then the direct epilogue's
+// steps: FP8 acc * (s_x[m] s_w[n]), INT8 fp32(acc) * fp32(s_x s_w) with each
+// step rounded once, + residual, bf16.  Outputs in 4-column groups over
+// `nthreads` threads, up to 16 splits' loads in flight per group.
+template <bool I8>
+__device__ __forceinline__ void splitk_finish_tile_8bit(const GemmArgs& a, int m_tile, int n_tile, int bn, int tid,
+                                                        int nthreads) {
+  constexpr int kLoads = 16;
+  const int r0 = m_tile * kBM, c0 = n_tile * bn;
+  const int rows = min(kBM, a.M - r0), cols = min(bn, a.N - c0);
+  const int groups = cols >> 2;  // N % 8 == 0
+  const size_t split_stride = static_cast<size_t>(a.M) * a.N;
+  for (int item = tid; item < rows * groups; item += nthreads) {
+    const int row = r0 + item / groups;
+    const int col = c0 + 4 * (item % groups);
+    const float* src = a.partial + static_cast<size_t>(row) * a.N + col;
+    float y[4];
+    if constexpr (I8) {
+      int acc[4] = {0, 0, 0, 0};
+      for (int sp = 0; sp < a.splits; sp += kLoads) {
+        int4 v[kLoads];
+#pragma unroll
+        for (int t = 0; t < kLoads; ++t)
+          v[t] = sp + t < a.splits ? __ldcg(reinterpret_cast<const int4*>(src + (sp + t) * split_stride))
+                                   : make_int4(0, 0, 0, 0);
+#pragma unroll
+        for (int t = 0; t < kLoads; ++t) {
+          acc[0] += v[t].x;
+          acc[1] += v[t].y;
+          acc[2] += v[t].z;
+          acc[3] += v[t].w;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) y[j] = int8_scaled(static_cast<uint32_t>(acc[j]), a.xg[row], a.wg[col + j]);
+    } else {
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      const float4 nz = make_float4(-0.0f, -0.0f, -0.0f, -0.0f);
+      for (int sp = 0; sp < a.splits; sp += kLoads) {
+        float4 v[kLoads];
+#pragma unroll
+        for (int t = 0; t < kLoads; ++t)
+          v[t] = sp + t < a.splits ? __ldcg(reinterpret_cast<const float4*>(src + (sp + t) * split_stride)) : nz;
+#pragma unroll
+        for (int t = 0; t < kLoads; ++t) {
+          acc[0] += v[t].x;
+          acc[1] += v[t].y;
+          acc[2] += v[t].z;
+          acc[3] += v[t].w;
+        }
+      }
+      const float rs = a.xg[row];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) y[j] = acc[j] * (rs * a.wg[col + j]);
+    }
+    const size_t o = static_cast<size_t>(row) * a.N + col;
+    if (a.residual) {
+      const uint2 rv = __ldg(reinterpret_cast<const uint2*>(a.residual + o));
+      y[0] = add_residual<I8>(y[0], __uint_as_float(rv.x << 16));
+      y[1] = add_residual<I8>(y[1], __uint_as_float(rv.x & 0xFFFF0000u));
+      y[2] = add_residual<I8>(y[2], __uint_as_float(rv.y << 16));
+      y[3] = add_residual<I8>(y[3], __uint_as_float(rv.y & 0xFFFF0000u));
+    }
+    *reinterpret_cast<uint2*>(a.Y + o) = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
+  }
+}
+
 // 8-bit W8A8 GEMM, FP8 E4M3 (kind::f8f6f4, fp32 accumulators) or INT8
 // (I8: kind::i8, exact s32 accumulators): 64 + 32 EPI_WARPS threads, warp 0
 // TMA producer, warp 1 TMEM allocator and MMA issuer, the rest epilogue
-// warps; split-K partials are added by splitk_reduce_kernel.
+// warps; the last split of a tile adds the split-K partials in-kernel.
 template <int BN, bool I8>
 __global__ void __launch_bounds__(Fp8Cfg<BN, I8>::THREADS, 1)
 gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -249,6 +324,7 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t s_tmem_base;
   __shared__ volatile int s_abort;
+  __shared__ int s_last;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
@@ -418,6 +494,24 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             store_partial(args, w.split, row, col0, r[c]);
           else
             store_output<false, I8>(args, row, col0, rs, r[c]);
+        }
+      }
+      if (args.splits > 1) {
+        // Split-K: the split that arrives last at the tile's counter adds
+        // the partials in split order and writes the output, then puts the
+        // counter back to zero for the next call (as in the NVFP4 kernel).
+        __threadfence();
+        named_bar_sync(1, 32 * C::EPI_WARPS);
+        if (e == 0 && lane == 0) {
+          unsigned int* cnt = args.counters + (w.n * args.m_tiles + w.m);
+          const unsigned int done = atomicAdd(cnt, 1u);
+          s_last = (done == static_cast<unsigned int>(args.splits - 1));
+          if (s_last) *cnt = 0u;
+        }
+        named_bar_sync(1, 32 * C::EPI_WARPS);
+        if (s_last) {
+          __threadfence();
+          splitk_finish_tile_8bit<I8>(args, w.m, w.n, BN, e * 32 + lane, 32 * C::EPI_WARPS);
         }
       }
     }
@@ -1339,60 +1433,6 @@ gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   }
 }
 
-// Split-K reduction + epilogue: fixed split order, same scaling as the
-// direct epilogue (INT8: exact s32 sums, then the INT8 epilogue steps).
-// 8 outputs per thread.
-template <bool FP4, bool I8 = false>
-__global__ void splitk_reduce_kernel(const float* __restrict__ partial, int splits, int M, int N,
-                                     const float* __restrict__ xg, const float* __restrict__ wg,
-                                     const __nv_bfloat16* __restrict__ residual,
-                                     __nv_bfloat16* __restrict__ Y) {
-  griddep_wait();
-  griddep_launch_dependents();
-  const int64_t idx8 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t total8 = static_cast<int64_t>(M) * N / 8;
-  if (idx8 >= total8) return;
-  const int64_t e0 = idx8 * 8;
-  const int row = static_cast<int>(e0 / N);
-  const int col = static_cast<int>(e0 % N);
-  float y[8];
-  if constexpr (I8) {
-    int acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int s = 0; s < splits; ++s) {
-      const int4* p = reinterpret_cast<const int4*>(partial + (static_cast<size_t>(s) * M) * N + e0);
-      const int4 a = p[0], b = p[1];
-      acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-      acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) y[j] = int8_scaled(static_cast<uint32_t>(acc[j]), xg[row], wg[col + j]);
-  } else {
-    float acc[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
-    for (int s = 0; s < splits; ++s) {
-      const float4* p = reinterpret_cast<const float4*>(partial + (static_cast<size_t>(s) * M) * N + e0);
-      const float4 a = p[0], b = p[1];
-      acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-      acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
-    }
-    const float rs = FP4 ? xg[row] * wg[0] : xg[row];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) y[j] = acc[j] * (FP4 ? rs : rs * wg[col + j]);
-  }
-  if (residual) {
-    const uint4 v = *reinterpret_cast<const uint4*>(residual + e0);
-    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      y[2 * t] = add_residual<I8>(y[2 * t], __uint_as_float(wv[t] << 16));
-      y[2 * t + 1] = add_residual<I8>(y[2 * t + 1], __uint_as_float(wv[t] & 0xFFFF0000u));
-    }
-  }
-  *reinterpret_cast<uint4*>(Y + e0) = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
-                                                 pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
-}
-
 // ------------------------------------------------------------ host side --
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -1734,7 +1774,7 @@ GemmArgs make_args(bool fp4, int BN, const uint8_t* xs, const float* xg, const u
   // split-K workspace: tile counters first (NVFP4), then the partial sums
   a.partial = plan.splits > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kSplitCounterBytes)
                               : nullptr;
-  a.counters = (fp4 && plan.splits > 1) ? static_cast<unsigned int*>(workspace) : nullptr;
+  a.counters = plan.splits > 1 ? static_cast<unsigned int*>(workspace) : nullptr;
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.K = static_cast<int>(K);
@@ -1897,14 +1937,7 @@ cudaError_t run_fp8(const uint8_t* xq, const float* xg, const uint8_t* wq, const
   auto kern = gemm_fp8_kernel<BN, I8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, s, ta, tb, a);
-  if (e != cudaSuccess || plan.splits == 1) return e;
-  const int64_t total8 = M * N / 8;
-  const int threads = 256;
-  const int64_t blocks = (total8 + threads - 1) / threads;
-  return launch_pdl(splitk_reduce_kernel<false, I8>, dim3(static_cast<unsigned int>(blocks)), dim3(threads), 0, s,
-                    static_cast<const float*>(a.partial), plan.splits, a.M, a.N, xg, wg,
-                    static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(Y));
+  return launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, s, ta, tb, a);
 }
 
 }  // namespace
